@@ -1,0 +1,75 @@
+// kernels.h -- launch interfaces between the host entry points and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gattn {
+
+struct PrefillArgs {
+  const int32_t* cu_seqlens;
+  void* out;
+  float* lse;
+  int num_seqs;
+  int max_qtiles;     // ceil(max_seqlen / 128)
+  int max_seqlen;
+  int total_tokens;
+  int num_q_heads;
+  int group;          // query heads per KV head
+  int head_dim;       // real head dim (row stride of out); the kernel dim may be padded to 64
+  int is_local;
+  int window;
+  float softmax_scale;
+  uint32_t rot_mask;  // bit c set: key/query chunk c (64 dims) is read from the rotated side copy
+};
+
+struct PrefillMaps {
+  CUtensorMap q, qs, k, ks, v;
+};
+
+template <int D>
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);
+
+// Rotated (or zero-padded) side copy of selected 64-dim chunks.
+struct RopeArgs {
+  const uint16_t* src;      // [T, H, d] bf16
+  uint16_t* dst;            // [T, H, n_out] bf16, n_out = popcount(chunk_mask) * 64
+  const int32_t* positions; // [T]
+  int tokens;
+  int heads;
+  int d;                    // real head dim
+  int r;                    // rotated pairs (0: copy only)
+  uint32_t chunk_mask;      // chunks of the (padded) head dim that are copied
+  int n_out;
+  double log2_base;
+};
+cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream);
+
+struct DecodeArgs {
+  const uint16_t* q;        // [B, n_q, Hq, d]
+  const uint16_t* new_k;    // [B, n_q, Hkv, d]
+  const uint16_t* new_v;    // [B, n_q, Hkv, d] or null (K=V)
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;  // null for K=V
+  const int32_t* cache_seqlens;
+  float* partial_o;         // [splits, rows, d]
+  float* partial_lse;       // [splits, rows]
+  int batch, n_q, num_q_heads, num_kv_heads, head_dim;
+  int is_local, window, ring, capacity, num_splits;
+  int r;
+  double log2_base;
+  float softmax_scale;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+struct CombineArgs {
+  const float* partial_o;
+  const float* partial_lse;
+  void* out;
+  float* lse;
+  int num_splits, rows, head_dim;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+}  // namespace gattn

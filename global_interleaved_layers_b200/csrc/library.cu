@@ -1,0 +1,7 @@
+// library.cu -- single translation unit for libgemma_attn.so, so that the device
+// status word and every kernel live in one module without relocatable device code.
+#include "api.cu"
+#include "rope.cu"
+#include "prefill.cu"
+#include "decode.cu"
+#include "selftest.cu"

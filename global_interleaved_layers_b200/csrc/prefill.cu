@@ -1,0 +1,382 @@
+// prefill.cu -- flash-style causal attention for Gemma-4-style local (sliding
+// window) and global (K=V, p-RoPE) layers on sm_100a.
+//
+// One CTA computes a 128-row query tile of one query head against the key tiles
+// its rows can see (global: all earlier keys; local: the last W keys; "Visual
+// guide to Gemma 4", section "Interleaving Layers"). Fully masked key tiles are
+// never loaded; only tiles that straddle the diagonal or the window edge are masked.
+//
+// Roles (192 threads):
+//   warp 0     TMA producer: the Q tile once, then 16 KB chunks (128 keys x 64
+//              dims, 128-byte swizzle) of K and V through a ring of stages.
+//   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score
+//              buffers (tcgen05.mma, both operands in shared memory), then
+//              O += P V with P read from TMEM and V from the ring.
+//   warps 2-5  softmax: one query row per thread; online softmax in fp32 with
+//              the running max only raised when it grows by more than 2^8, P written
+//              back to TMEM as bf16 over the scores, epilogue O / l -> bf16.
+// The MMA order is S(j), PV(j-1), S(j+1), PV(j), ... so the tensor core works on
+// S(j+1) while the softmax warps turn S(j) into P(j).
+//
+// Global layers: the single K=V tensor feeds both operands. Key chunks that hold
+// rotated dimensions come from a rotated side copy (workspace); every other key
+// chunk and every value chunk are read from the un-rotated tensor ("Visual guide
+// to Gemma 4", sections "K=V technique" and "p-RoPE"). With head_dim 512 the
+// 128 x 512 fp32 output tile would fill all of TMEM, so two CTAs each own one
+// 256-column half of the output and both compute the full score tile.
+#include "common.cuh"
+#include "kernels.h"
+#include "tile_plan.h"
+
+namespace gattn {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kChunk = 64;                   // dims per TMA box / swizzle row
+constexpr int kStageBytes = kBN * 128;       // 128 rows x 128 bytes
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kDv = D > 256 ? 256 : D;             // output columns per CTA
+  static constexpr int kSplit = D / kDv;                      // CTAs per (tile, head)
+  static constexpr int kQChunks = D / kChunk;
+  static constexpr int kVChunks = kDv / kChunk;
+  static constexpr int kQBytes = kQChunks * kStageBytes;
+  static constexpr int kStages = D >= 512 ? 6 : 8;
+  static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct __align__(8) Barriers {
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done;
+  uint64_t mma_done;
+  uint64_t ring_full[8];
+  uint64_t ring_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap qs_map,
+               const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap ks_map,
+               const __grid_constant__ CUtensorMap v_map, PrefillArgs args) {
+  using Cfg = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;
+  uint8_t* ring = smem + Cfg::kQBytes;
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + Cfg::kSmemData);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- which work unit ----
+  const int head = blockIdx.x / Cfg::kSplit;
+  const int vpart = blockIdx.x % Cfg::kSplit;
+  const int slot = blockIdx.y;
+  const int seq = slot % args.num_seqs;
+  const int qt = args.max_qtiles - 1 - slot / args.num_seqs;  // heaviest tiles first
+  const int tok0 = args.cu_seqlens[seq];
+  const int len = args.cu_seqlens[seq + 1] - tok0;
+  if (qt == 0 && vpart == 0 && head == 0 && threadIdx.x == 0 && (len > args.max_seqlen || len < 1))
+    atomicOr(&g_status, kStatusSeqlen);
+  if (qt * kBM >= len) return;
+  const int row0 = qt * kBM;
+  const int kvh = head / args.group;
+  const int is_local = args.is_local;
+  int kt_lo, kt_hi;
+  kv_tile_range(is_local, args.window, len, qt, kBM, kBN, &kt_lo, &kt_hi);
+  const int ntiles = kt_hi - kt_lo;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->s_full[b], 1); mbar_init(&bars->p_full[b], 128); }
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->mma_done, 1);
+    for (int s = 0; s < Cfg::kStages; ++s) { mbar_init(&bars->ring_full[s], 1); mbar_init(&bars->ring_empty[s], 1); }
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&q_map); prefetch_tensormap(&k_map); prefetch_tensormap(&v_map);
+      if (args.rot_mask) { prefetch_tensormap(&qs_map); prefetch_tensormap(&ks_map); }
+      mbar_arrive_expect_tx(&bars->q_full, Cfg::kQBytes);
+      for (int c = 0; c < Cfg::kQChunks; ++c) {
+        if ((args.rot_mask >> c) & 1) {
+          int ridx = __popc(args.rot_mask & ((1u << c) - 1));
+          tma_load_3d(q_smem + c * kStageBytes, &qs_map, &bars->q_full, ridx * kChunk, head, tok0 + row0);
+        } else {
+          tma_load_3d(q_smem + c * kStageBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
+        }
+      }
+      int st = 0; uint32_t ph = 0;
+      auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
+      bool ok = true;
+      for (int jj = 0; jj <= ntiles && ok; ++jj) {
+        if (jj < ntiles) {  // K chunks of tile jj
+          const int key0 = tok0 + (kt_lo + jj) * kBN;
+          for (int c = 0; c < Cfg::kQChunks && ok; ++c) {
+            ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&bars->ring_full[st], kStageBytes);
+            if ((args.rot_mask >> c) & 1) {
+              int ridx = __popc(args.rot_mask & ((1u << c) - 1));
+              tma_load_3d(ring + st * kStageBytes, &ks_map, &bars->ring_full[st], ridx * kChunk, kvh, key0);
+            } else {
+              tma_load_3d(ring + st * kStageBytes, &k_map, &bars->ring_full[st], c * kChunk, kvh, key0);
+            }
+            next();
+          }
+        }
+        if (jj >= 1) {  // V chunks of tile jj-1 (this CTA's output columns)
+          const int key0 = tok0 + (kt_lo + jj - 1) * kBN;
+          for (int c = 0; c < Cfg::kVChunks && ok; ++c) {
+            ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&bars->ring_full[st], kStageBytes);
+            tma_load_3d(ring + st * kStageBytes, &v_map, &bars->ring_full[st],
+                        vpart * Cfg::kDv + c * kChunk, kvh, key0);
+            next();
+          }
+        }
+      }
+      // Let every copy this thread issued land before the CTA can exit: the last
+      // kStages loads are the only ones that may still be in flight.
+      for (int s = 0; s < Cfg::kStages; ++s) {
+        if (!mbar_try_wait(&bars->ring_full[st], ph)) {
+          unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&bars->ring_full[st], ph) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+        }
+        next();
+        (void)s;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(kBM, kBN, 0, 0);
+      const uint32_t idesc_pv = umma_idesc_bf16(kBM, kChunk, 0, 1);
+      const uint32_t q_base = smem_u32(q_smem);
+      const uint32_t r_base = smem_u32(ring);
+      int st = 0; uint32_t ph = 0;
+      auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
+      for (int jj = 0; jj <= ntiles && ok; ++jj) {
+        if (jj < ntiles) {
+          const int b = jj & 1;
+          const uint32_t s_col = b ? kColS1 : kColS0;
+          if (jj >= 2) ok = mbar_wait(&bars->pv_done, (uint32_t)(jj - 2) & 1u, abort_flag);
+          tc_fence_after();
+          for (int c = 0; c < Cfg::kQChunks && ok; ++c) {
+            ok = mbar_wait(&bars->ring_full[st], ph, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk) {
+              uint64_t a = sdesc_sw128(q_base + c * kStageBytes + kk * 32, 16, 1024);
+              uint64_t bdesc = sdesc_sw128(r_base + st * kStageBytes + kk * 32, 16, 1024);
+              umma_ss(tmem + s_col, a, bdesc, idesc_qk, (c | kk) != 0);
+            }
+            umma_commit(&bars->ring_empty[st]);
+            next();
+          }
+          if (!ok) break;
+          umma_commit(&bars->s_full[b]);
+        }
+        if (jj >= 1) {
+          const int pj = jj - 1;
+          const int pb = pj & 1;
+          const uint32_t p_col = pb ? kColS1 : kColS0;
+          ok = mbar_wait(&bars->p_full[pb], (uint32_t)(pj >> 1) & 1u, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          for (int c = 0; c < Cfg::kVChunks && ok; ++c) {
+            ok = mbar_wait(&bars->ring_full[st], ph, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              uint64_t bdesc = sdesc_sw128(r_base + st * kStageBytes + kk * 2048, kStageBytes, 1024);
+              umma_ts(tmem + kColO + c * kChunk, tmem + p_col + kk * 8, bdesc, idesc_pv, (pj | kk) != 0);
+            }
+            umma_commit(&bars->ring_empty[st]);
+            next();
+          }
+          if (!ok) break;
+          umma_commit(&bars->pv_done);
+        }
+      }
+      // All MMAs issued by this thread are complete once mma_done fires.
+      umma_commit(&bars->mma_done);
+      unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(&bars->mma_done, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float scale_log2 = args.softmax_scale * 1.4426950408889634f;
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    const int grow = row0 + row;  // in-sequence offset of this thread's query row
+    bool ok = true;
+    for (int jj = 0; jj < ntiles && ok; ++jj) {
+      const int b = jj & 1;
+      const uint32_t s_col = b ? kColS1 : kColS0;
+      ok = mbar_wait(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      float t[kBN];
+      uint32_t* tr = reinterpret_cast<uint32_t*>(t);
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
+      tmem_ld_wait();
+      const int kt = kt_lo + jj;
+      const bool partial = kv_tile_class(is_local, args.window, len, qt, kt, kBM, kBN) != kTileFull;
+      float m_tile = -INFINITY;
+      if (partial) {
+        const int k0 = kt * kBN;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          const int key = k0 + c;
+          const bool vis = key <= grow && (!is_local || key > grow - args.window);
+          t[c] = vis ? t[c] * scale_log2 : -INFINITY;
+          m_tile = fmaxf(m_tile, t[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          t[c] *= scale_log2;
+          m_tile = fmaxf(m_tile, t[c]);
+        }
+      }
+      // O may only be touched once PV(jj-1) has finished.
+      if (jj >= 1) {
+        ok = mbar_wait(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (m_tile > m_used + kRescaleThreshold || (m_used == -INFINITY && m_tile > -INFINITY)) {
+        if (m_used != -INFINITY) {
+          const float alpha = fast_exp2(m_used - m_tile);
+          l_sum *= alpha;
+          // rescale this row of O (written by PV(0..jj-1))
+#pragma unroll 1
+          for (int c = 0; c < Cfg::kDv / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
+          }
+        }
+        m_used = m_tile;
+      }
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+      uint32_t p[kBN / 2];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN / 2; ++c) {
+        float p0 = fast_exp2(t[2 * c] - m_sub);
+        float p1 = fast_exp2(t[2 * c + 1] - m_sub);
+        rs += p0 + p1;
+        p[c] = pack_bf16x2(p0, p1);
+      }
+      l_sum += rs;
+      tmem_st_x32(tmem + lane_off + s_col, p);
+      tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[b]);
+    }
+    if (ok && ntiles > 0) ok = mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      const bool valid = grow < len;
+      const int tok = tok0 + grow;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) +
+                            ((size_t)tok * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv;
+#pragma unroll 1
+      for (int c = 0; c < Cfg::kDv / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
+        tmem_ld_wait();
+        if (valid && vpart * Cfg::kDv + c * 32 < args.head_dim) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (valid && vpart == 0 && args.lse != nullptr)
+        args.lse[(size_t)head * args.total_tokens + tok] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+int prefill_smem_bytes() { return PrefillCfg<D>::kSmemBytes; }
+
+template <int D>
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
+  using Cfg = PrefillCfg<D>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(args.num_q_heads * Cfg::kSplit, args.num_seqs * args.max_qtiles);
+  prefill_kernel<D><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(maps.q, maps.qs, maps.k, maps.ks, maps.v, args);
+  return cudaGetLastError();
+}
+
+int prefill_out_split(int D) { return D > 256 ? D / 256 : 1; }
+
+template cudaError_t launch_prefill<64>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);
+template cudaError_t launch_prefill<128>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);
+template cudaError_t launch_prefill<256>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);
+template cudaError_t launch_prefill<512>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);
+
+}  // namespace gattn

@@ -1,0 +1,193 @@
+/*
+ * gemma_attn.h -- C ABI of the B200 (sm_100a) attention kernels for
+ * Gemma-4-style interleaved layers.
+ *
+ * Two layer kinds, as described in "Visual guide to Gemma 4":
+ *   LOCAL  -- sliding-window causal attention (section "Interleaving Layers":
+ *             a local layer looks only at tokens within a fixed range), with
+ *             grouped-query attention (2 query heads per KV head on local
+ *             layers per the DeepMind talk summary, section "Optimised
+ *             attention: local and global layers"), separate K and V.
+ *   GLOBAL -- full causal attention (same sections: a global layer sees the whole
+ *             preceding sequence) with GQA (8 query heads per KV head, guide
+ *             section "GQA"), K = V (guide section "K=V technique": one stored
+ *             tensor per KV head serves as keys and values) and p-RoPE (guide
+ *             section "p-RoPE": only the highest-frequency fraction p of the
+ *             rotary pairs is rotated; the rest pass through).
+ *
+ * Conventions shared by every entry point:
+ *   - bf16 tensors are passed as device pointers to raw bfloat16 storage; LSE and
+ *     split partials are float32; positions and lengths are int32.
+ *   - Head layout of q/k/v/out is row-major [tokens, heads, head_dim].
+ *   - Visible keys of a query at position i: pos_k <= i (GLOBAL) and additionally
+ *     pos_k > i - window (LOCAL): exactly `window` keys including the query itself.
+ *   - Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   - Rotary embedding: r = floor(rope_p * head_dim / 2) pairs (j, j + head_dim/2),
+ *     j = 0 .. r-1, rotated counter-clockwise by pos * rope_base^(-2j/head_dim).
+ *     q and the key copy used for scores are rotated; values never are (for
+ *     GLOBAL the single K=V tensor is stored un-rotated).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream). The caller owns every buffer, including
+ *     workspaces; the library allocates no device memory.
+ *   - Return value: GEMMA_ATTN_OK (0) or a negative status. On an argument error
+ *     nothing is launched. Device-side failures (a bounded wait that ran out, a
+ *     sequence longer than the stated maximum) are recorded in a device status
+ *     word that gemma_attn_check() reads and clears.
+ *   - Pointers to bf16 tensors read by the tensor-memory-accelerator loads must be
+ *     16-byte aligned; head_dim * 2 bytes must be a multiple of 16.
+ */
+#ifndef GEMMA_ATTN_H_
+#define GEMMA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  GEMMA_ATTN_LOCAL = 0,
+  GEMMA_ATTN_GLOBAL = 1
+};
+
+enum {
+  GEMMA_ATTN_CACHE_CONTIGUOUS = 0, /* [batch, kv_heads, capacity, head_dim]; token p at row p */
+  GEMMA_ATTN_CACHE_RING = 1        /* [batch, kv_heads, window, head_dim]; token p at slot p mod window */
+};
+
+enum {
+  GEMMA_ATTN_OK = 0,
+  GEMMA_ATTN_ERR_INVALID_ARG = -1,
+  GEMMA_ATTN_ERR_UNSUPPORTED = -2,
+  GEMMA_ATTN_ERR_WORKSPACE = -3,
+  GEMMA_ATTN_ERR_MISALIGNED = -4,
+  GEMMA_ATTN_ERR_LAUNCH = -5,
+  GEMMA_ATTN_ERR_TIMEOUT = -6,
+  GEMMA_ATTN_ERR_DEVICE = -7,
+  GEMMA_ATTN_ERR_SEQLEN = -8
+};
+
+/* Layer description. head_dim in {32, 64, 128, 256, 512}; num_q_heads a multiple of
+ * num_kv_heads; window >= 1 for LOCAL (ignored for GLOBAL); 0 <= rope_p <= 1;
+ * rope_base > 0; softmax_scale > 0 (typically 1/sqrt(head_dim)). */
+typedef struct gemma_attn_params {
+  int32_t kind;
+  int32_t window;
+  float rope_p;
+  float rope_base;
+  float softmax_scale;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+} gemma_attn_params;
+
+/* Bytes of device workspace gemma_attn_prefill needs for `total_tokens` tokens
+ * (a rotated copy of the key columns that p-RoPE touches, and of small heads'
+ * operands padded to 64 dims). Written to *bytes. */
+int gemma_attn_prefill_workspace_size(const gemma_attn_params* params, int32_t total_tokens,
+                                      size_t* bytes);
+
+/*
+ * Prefill: attention of every token of a ragged batch against the earlier tokens
+ * of its own sequence (flash-style; fully masked key tiles are never visited, so a
+ * LOCAL layer costs O(tokens * window)).
+ *   q         [total_tokens, num_q_heads, head_dim] bf16, device.
+ *   k         [total_tokens, num_kv_heads, head_dim] bf16, device (GLOBAL: the K=V tensor).
+ *   v         same shape as k for LOCAL; must be NULL for GLOBAL (values = k, un-rotated).
+ *   out       [total_tokens, num_q_heads, head_dim] bf16, device, written.
+ *   lse       [num_q_heads, total_tokens] float32 natural-log sum-exp of the scaled
+ *             scores, device, written; may be NULL.
+ *   positions [total_tokens] int32, device: rotary position of each token. Within a
+ *             sequence the positions must be consecutive (p, p+1, ...): the masks are
+ *             evaluated on in-sequence offsets, which equals the position rule then.
+ *   cu_seqlens [num_seqs + 1] int32, device: sequence s is tokens cu[s] .. cu[s+1]-1.
+ *             Lengths must be >= 1 and <= max_seqlen (violations are reported through
+ *             gemma_attn_check as GEMMA_ATTN_ERR_SEQLEN).
+ *   workspace  device buffer of at least gemma_attn_prefill_workspace_size() bytes,
+ *             256-byte aligned; contents are scratch.
+ */
+int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const void* k, const void* v,
+                       void* out, float* lse, const int32_t* positions, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode / speculative verify, split-KV stage: n_q new query tokens per sequence
+ * attend to that sequence's cache plus the new tokens themselves.
+ *   q          [batch, n_q, num_q_heads, head_dim] bf16; query i of sequence b sits at
+ *              position cache_seqlens[b] + i.
+ *   new_k      [batch, n_q, num_kv_heads, head_dim] bf16: keys of the new tokens
+ *              (GLOBAL: their K=V rows). Required (n_q >= 1).
+ *   new_v      same shape for LOCAL; NULL for GLOBAL.
+ *   k_cache    GEMMA_ATTN_CACHE_CONTIGUOUS: [batch, num_kv_heads, cache_capacity, head_dim],
+ *              token p of sequence b at row p (p < cache_seqlens[b] <= cache_capacity).
+ *              GEMMA_ATTN_CACHE_RING (LOCAL only): [batch, num_kv_heads, window, head_dim],
+ *              token p at slot p mod window, holding the last min(len, window) tokens;
+ *              cache_capacity must equal window.
+ *              Caches hold un-rotated keys (GLOBAL: the K=V tensor).
+ *   v_cache    same layout as k_cache for LOCAL; NULL for GLOBAL.
+ *   cache_seqlens [batch] int32 device: tokens already cached (>= 0).
+ *   max_cache_len  upper bound on cache_seqlens (sizes the launch).
+ *   partial_o  [num_splits, batch * n_q * num_q_heads, head_dim] float32, written.
+ *   partial_lse [num_splits, batch * n_q * num_q_heads] float32, written (-inf for an
+ *              empty split). Row index = (b * n_q + i) * num_q_heads + h.
+ *   The visible keys of each sequence are cut into num_splits contiguous ranges.
+ */
+int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void* new_k,
+                      const void* new_v, const void* k_cache, const void* v_cache,
+                      int32_t cache_layout, int32_t cache_capacity, const int32_t* cache_seqlens,
+                      int32_t batch, int32_t n_q, int32_t max_cache_len,
+                      float* partial_o, float* partial_lse, int32_t num_splits, void* stream);
+
+/* A split count for gemma_attn_decode that fills the GPU for this shape. */
+int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,
+                                 int32_t max_cache_len, int32_t* num_splits);
+
+/*
+ * Combine split partials: out = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M) with
+ * M = max_s lse_s; lse = M + log(sum_s exp(lse_s - M)).
+ *   partial_o [num_splits, rows, head_dim] f32, partial_lse [num_splits, rows] f32 (device).
+ *   out [rows, head_dim] bf16 (device, written); lse [rows] f32 or NULL.
+ */
+int gemma_attn_combine(const float* partial_o, const float* partial_lse, int32_t num_splits,
+                       int32_t rows, int32_t head_dim, void* out, float* lse, void* stream);
+
+/*
+ * Host-side tile plan (the same rule the prefill kernels apply): for every sequence,
+ * query tile of bm rows and key tile of bn keys with at least one visible pair, one
+ * 4-tuple (sequence, q_tile, kv_tile, class) with class 1 = partially masked,
+ * 2 = fully visible, ordered by sequence, q_tile, kv_tile. cu_seqlens is HOST memory.
+ * Writes min(cap, count) tuples to out (may be NULL) and the count to *count.
+ */
+int gemma_attn_tile_plan(int32_t kind, int32_t window, const int32_t* cu_seqlens_host,
+                         int32_t num_seqs, int32_t bm, int32_t bn, int32_t* out, int64_t cap,
+                         int64_t* count);
+
+/* Synchronise `stream`, return (and clear) the device status word: GEMMA_ATTN_OK,
+ * GEMMA_ATTN_ERR_TIMEOUT or GEMMA_ATTN_ERR_SEQLEN; GEMMA_ATTN_ERR_DEVICE on a CUDA error. */
+int gemma_attn_check(void* stream);
+
+/* Static description of a status code. */
+const char* gemma_attn_error_string(int status);
+
+/* Number of kernel launches the last successful call on this host thread issued. */
+int gemma_attn_last_launch_count(void);
+
+/*
+ * Diagnostic: one 128-row tile through each tensor-core operand form the prefill
+ * kernel uses, for tests that recompute the product on the host. Device pointers:
+ *   mode 0: a [128][128] bf16, b [128][128] bf16 (both K-major in shared memory);
+ *           d [128][128] f32 = a * b^T.
+ *   mode 1: p [128][128] bf16 staged through tensor memory, b [128][64] bf16 read
+ *           MN-major; d [128][64] f32 = p * b.
+ * a must be NULL-or-ignored in mode 1 and p in mode 0.
+ */
+int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const void* p, float* d,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GEMMA_ATTN_H_ */

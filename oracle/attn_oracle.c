@@ -53,20 +53,34 @@ int oracle_rotated_pairs(double rope_p, int head_dim) {
   return (int)floor(rope_p * (double)head_dim / 2.0);
 }
 
-/* Rotate x (length d) for position pos: pairs (j, j + d/2), j < r, angle pos * base^(-2j/d).
- * The other coordinates are copied unchanged. */
-void oracle_rope(const double* x, double* y, int d, double rope_p, double rope_base, double pos) {
+/* cos and sin of the rotation angle pos * base^(-2j/d) for pair j. */
+static void rope_angle(double pos, int j, int d, double rope_base, double* c, double* s) {
+  double theta = pow(rope_base, -2.0 * (double)j / (double)d);
+  double a = pos * theta;
+  *c = cos(a);
+  *s = sin(a);
+}
+
+/* Rotate x (length d) given cos/sin of each rotated pair: pairs (j, j + d/2), j < r,
+ * counter-clockwise. The other coordinates are copied unchanged. */
+static void rope_apply(const double* x, double* y, int d, int r, const double* cs) {
   int half = d / 2;
-  int r = oracle_rotated_pairs(rope_p, d);
   for (int i = 0; i < d; ++i) y[i] = x[i];
   for (int j = 0; j < r; ++j) {
-    double theta = pow(rope_base, -2.0 * (double)j / (double)d);
-    double a = pos * theta;
-    double c = cos(a), s = sin(a);
+    double c = cs[2 * j], s = cs[2 * j + 1];
     double x0 = x[j], x1 = x[j + half];
     y[j] = x0 * c - x1 * s;
     y[j + half] = x0 * s + x1 * c;
   }
+}
+
+/* Rotate x (length d) for position pos. */
+void oracle_rope(const double* x, double* y, int d, double rope_p, double rope_base, double pos) {
+  int r = oracle_rotated_pairs(rope_p, d);
+  double* cs = (double*)malloc(sizeof(double) * 2 * (r > 0 ? r : 1));
+  for (int j = 0; j < r; ++j) rope_angle(pos, j, d, rope_base, &cs[2 * j], &cs[2 * j + 1]);
+  rope_apply(x, y, d, r, cs);
+  free(cs);
 }
 
 static int seq_of_token(const int32_t* cu_seqlens, int num_seqs, int t) {
@@ -105,6 +119,23 @@ int oracle_attention(int kind, int window, double rope_p, double rope_base, doub
   const uint16_t* vv = v ? v : k;
   int T = cu_seqlens[num_seqs];
   if (!rows) n_rows = T;
+  const int r = oracle_rotated_pairs(rope_p, d);
+
+  /* cos/sin of every (position, pair) that occurs, computed once: the same values
+   * rope_angle would return at each use. */
+  int pmin = 0, pmax = 0;
+  for (int t = 0; t < T; ++t) {
+    if (t == 0 || positions[t] < pmin) pmin = positions[t];
+    if (t == 0 || positions[t] > pmax) pmax = positions[t];
+  }
+  const long long npos = (long long)pmax - pmin + 1;
+  const int rr = r > 0 ? r : 1;
+  double* table = (double*)malloc(sizeof(double) * 2 * (size_t)rr * (size_t)npos);
+  if (!table) return -2;
+#pragma omp parallel for schedule(static)
+  for (long long pi = 0; pi < npos; ++pi)
+    for (int j = 0; j < r; ++j)
+      rope_angle((double)(pmin + pi), j, d, rope_base, &table[(pi * rr + j) * 2], &table[(pi * rr + j) * 2 + 1]);
 
   long long jobs = (long long)n_rows * Hq;
 #pragma omp parallel
@@ -125,7 +156,7 @@ int oracle_attention(int kind, int window, double rope_p, double rope_base, doub
       int g = h / group;
       if (end - beg > cap) { cap = end - beg; z = (double*)realloc(z, sizeof(double) * cap); }
       for (int i = 0; i < d; ++i) qv[i] = bf16_to_double(q[((size_t)t * Hq + h) * d + i]);
-      oracle_rope(qv, qr, d, rope_p, rope_base, (double)positions[t]);
+      rope_apply(qv, qr, d, r, &table[(size_t)(positions[t] - pmin) * rr * 2]);
       /* scores of visible keys */
       double zmax = -INFINITY;
       int any = 0;
@@ -135,7 +166,7 @@ int oracle_attention(int kind, int window, double rope_p, double rope_base, doub
         if (key_hi > key_lo && (idx < key_lo || idx >= key_hi)) continue;
         if (!key_visible(kind, window, positions[t], positions[u])) continue;
         for (int i = 0; i < d; ++i) kv[i] = bf16_to_double(k[((size_t)u * Hkv + g) * d + i]);
-        oracle_rope(kv, kr, d, rope_p, rope_base, (double)positions[u]);
+        rope_apply(kv, kr, d, r, &table[(size_t)(positions[u] - pmin) * rr * 2]);
         double dot = 0.0;
         for (int i = 0; i < d; ++i) dot += qr[i] * kr[i];
         z[idx] = scale * dot;
@@ -163,6 +194,7 @@ int oracle_attention(int kind, int window, double rope_p, double rope_base, doub
     }
     free(qv); free(qr); free(kv); free(kr); free(acc); free(z);
   }
+  free(table);
   return 0;
 }
 

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path (called through the C-ABI) against the fp64 oracle.
+
+Bounds (from the acceptance criteria): max-abs <= 1e-2 and relative RMS <= 5e-3 on
+outputs; lse within 1e-2. Shapes span several 128-row tiles with ragged tails, GQA
+ratios 2:1 and 8:1, head dims 32..512, windows from 1 to beyond the length,
+K=V with p-RoPE, and position offsets.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+G = pytest.importorskip("global_interleaved_layers_b200")
+from gpu_util import assert_close, dev_bf16, dev_i32, host_bits, ring_from_history, run_prefill  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def _bf16_to_f64(bits):
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ------------------------------------------------------------------ tensor-core operand forms
+
+def test_umma_selftest_ss_kmajor():
+    rng = np.random.default_rng(1)
+    a = W.f32_to_bf16_bits(rng.standard_normal((128, 128), dtype=np.float32))
+    b = W.f32_to_bf16_bits(rng.standard_normal((128, 128), dtype=np.float32))
+    d = torch.zeros((128, 128), dtype=torch.float32, device="cuda")
+    G.gemma_attn_selftest_umma(0, dev_bf16(a), dev_bf16(b), None, d)
+    torch.cuda.synchronize()
+    ref = _bf16_to_f64(a) @ _bf16_to_f64(b).T
+    np.testing.assert_allclose(d.cpu().numpy(), ref, rtol=1e-4, atol=1e-3)
+
+
+def test_umma_selftest_ts_mnmajor():
+    rng = np.random.default_rng(2)
+    p = W.f32_to_bf16_bits(rng.standard_normal((128, 128), dtype=np.float32))
+    v = W.f32_to_bf16_bits(rng.standard_normal((128, 64), dtype=np.float32))
+    d = torch.zeros((128, 64), dtype=torch.float32, device="cuda")
+    G.gemma_attn_selftest_umma(1, None, dev_bf16(v), dev_bf16(p), d)
+    torch.cuda.synchronize()
+    ref = _bf16_to_f64(p) @ _bf16_to_f64(v)
+    np.testing.assert_allclose(d.cpu().numpy(), ref, rtol=1e-4, atol=1e-3)
+
+
+# ------------------------------------------------------------------ prefill
+
+def _check_prefill(layer, seq_lens, seed=0, pos_start=0, rows=None):
+    T = int(sum(seq_lens))
+    q, k, v = W.layer_inputs(layer, T, seed)
+    cu = np.concatenate([[0], np.cumsum(seq_lens)]).astype(np.int32)
+    pos = np.concatenate([np.arange(n) + pos_start for n in seq_lens]).astype(np.int32)
+    out, lse = run_prefill(G, layer, q, k, v, pos, cu)
+    got = W.bf16_bits_to_f32(host_bits(out))
+    got_lse = lse.cpu().numpy()
+    ref, ref_lse = oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                                    q, k, v, pos, cu, rows=rows)
+    if rows is not None:
+        got = got[rows]
+        got_lse = got_lse[:, rows]
+    assert_close(got, ref, f"prefill {layer} lens={seq_lens}")
+    np.testing.assert_allclose(got_lse.T, ref_lse, atol=1e-2, rtol=0)
+
+
+def test_prefill_tiny_config_both_layers():
+    wl = W.tiny_ref()
+    for layer in wl.layers:
+        _check_prefill(layer, wl.seq_lens, seed=wl.seed)
+
+
+@pytest.mark.parametrize("layer,lens", [
+    (W.LayerSpec(W.LOCAL, 4, 2, 256, window=300, rope_p=1.0, rope_base=1e4), (700,)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 256, window=512, rope_p=1.0, rope_base=1e4), (1, 129, 300, 513)),
+    (W.LayerSpec(W.LOCAL, 2, 1, 256, window=1, rope_p=1.0, rope_base=1e4), (257,)),
+    (W.LayerSpec(W.LOCAL, 2, 1, 256, window=5000, rope_p=1.0, rope_base=1e4), (300,)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 128, window=200, rope_p=1.0, rope_base=1e4), (450,)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 64, window=100, rope_p=0.5, rope_base=1e4), (333,)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 32, window=40, rope_p=1.0, rope_base=1e4), (200, 77)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6), (600,)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6), (1, 200, 257)),
+    (W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.0, rope_base=1e6), (300,)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 256, rope_p=0.25, rope_base=1e4), (390,)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 64, rope_p=0.25, rope_base=1e4), (260,)),
+])
+def test_prefill_shapes(layer, lens):
+    _check_prefill(layer, lens, seed=3)
+
+
+def test_prefill_position_offset():
+    layer = W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
+    _check_prefill(layer, (300,), seed=4, pos_start=100000)
+    layer = W.LayerSpec(W.LOCAL, 4, 2, 256, window=128, rope_p=1.0, rope_base=1e4)
+    _check_prefill(layer, (300,), seed=5, pos_start=60000)
+
+
+def test_prefill_seqlen_violation_reported():
+    layer = W.LayerSpec(W.LOCAL, 2, 1, 64, window=16)
+    q, k, v = W.layer_inputs(layer, 300, 0)
+    p = G.params(layer.kind, 2, 1, 64, window=16)
+    ws_bytes = G.gemma_attn_prefill_workspace_size(p, 300)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    out = torch.empty((300, 2, 64), dtype=torch.bfloat16, device="cuda")
+    G.gemma_attn_prefill(p, dev_bf16(q), dev_bf16(k), dev_bf16(v), out, None, dev_i32(np.arange(300)),
+                         dev_i32([0, 300]), 1, 300, 100, ws, ws_bytes)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_check()
+    assert e.value.status == G.ERR_SEQLEN
+    G.gemma_attn_check()  # cleared
+
+
+# ------------------------------------------------------------------ decode / verify + combine
+
+def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11):
+    B = len(cache_lens)
+    Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+    rng_seed = seed
+    k_hist, v_hist = [], []
+    for b, n in enumerate(cache_lens):
+        k_hist.append(W.normal_bf16(rng_seed + 100 * b, 1, (n + n_q, Hkv, d)))
+        v_hist.append(None if layer.k_eq_v else W.normal_bf16(rng_seed + 100 * b, 2, (n + n_q, Hkv, d)))
+    q = W.normal_bf16(rng_seed, 0, (B, n_q, Hq, d))
+    ref, ref_lse = oracle.decode(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                                 q, k_hist, None if layer.k_eq_v else v_hist, cache_lens)
+    max_len = max(cache_lens)
+    if layout == G.CACHE_RING:
+        cap = layer.window
+        kc = np.stack([ring_from_history(k_hist[b][:cache_lens[b]], cap) for b in range(B)])
+        vc = None if layer.k_eq_v else np.stack([ring_from_history(v_hist[b][:cache_lens[b]], cap) for b in range(B)])
+    else:
+        cap = max(max_len, 1)
+        kc = np.zeros((B, Hkv, cap, d), np.uint16)
+        vc = None if layer.k_eq_v else np.zeros((B, Hkv, cap, d), np.uint16)
+        for b, n in enumerate(cache_lens):
+            kc[b, :, :n] = k_hist[b][:n].transpose(1, 0, 2)
+            if vc is not None:
+                vc[b, :, :n] = v_hist[b][:n].transpose(1, 0, 2)
+    new_k = np.stack([k_hist[b][cache_lens[b]:] for b in range(B)])
+    new_v = None if layer.k_eq_v else np.stack([v_hist[b][cache_lens[b]:] for b in range(B)])
+    p = G.params(layer.kind, Hq, Hkv, d, window=layer.window, rope_p=layer.rope_p, rope_base=layer.rope_base,
+                 softmax_scale=layer.softmax_scale)
+    if num_splits is None:
+        num_splits = G.gemma_attn_decode_num_splits(p, B, n_q, max_len)
+    rows = B * n_q * Hq
+    po = torch.empty((num_splits, rows, d), dtype=torch.float32, device="cuda")
+    pl = torch.empty((num_splits, rows), dtype=torch.float32, device="cuda")
+    G.gemma_attn_decode(p, dev_bf16(q), dev_bf16(new_k), None if new_v is None else dev_bf16(new_v), dev_bf16(kc),
+                        None if vc is None else dev_bf16(vc), layout, cap, dev_i32(cache_lens), B, n_q, max_len,
+                        po, pl, num_splits)
+    out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    G.gemma_attn_combine(po, pl, num_splits, rows, d, out, lse)
+    G.gemma_attn_check()
+    got = W.bf16_bits_to_f32(host_bits(out))
+    assert_close(got, ref, f"decode {layer} lens={cache_lens} n_q={n_q} splits={num_splits}")
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(ref_lse.shape), ref_lse, atol=1e-2, rtol=0)
+
+
+LOC = W.LayerSpec(W.LOCAL, 8, 4, 256, window=64, rope_p=1.0, rope_base=1e4)
+GLO = W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.25, rope_base=1e6)
+
+
+@pytest.mark.parametrize("cache_lens,n_q,splits", [
+    ((0, 5, 63, 64, 200), 1, None),
+    ((1000, 130), 1, 3),
+    ((77, 300), 4, 1),
+    ((77, 300), 4, 5),
+])
+def test_decode_local_ring(cache_lens, n_q, splits):
+    _check_decode(LOC, cache_lens, n_q, G.CACHE_RING, splits)
+
+
+def test_decode_local_contiguous():
+    _check_decode(LOC, (10, 250), 2, G.CACHE_CONTIGUOUS, 4)
+
+
+@pytest.mark.parametrize("cache_lens,n_q,splits", [
+    ((0, 1, 300), 1, None),
+    ((2000, 513), 1, 7),
+    ((150, 400), 4, 3),
+])
+def test_decode_global(cache_lens, n_q, splits):
+    _check_decode(GLO, cache_lens, n_q, G.CACHE_CONTIGUOUS, splits)
+
+
+def test_decode_global_gqa8():
+    _check_decode(W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6), (1500,), 1, G.CACHE_CONTIGUOUS)
+
+
+def test_combine_against_oracle():
+    rng = np.random.default_rng(9)
+    S, R, d = 5, 37, 64
+    po = rng.standard_normal((S, R, d)).astype(np.float32)
+    pl = (rng.standard_normal((S, R)) * 3).astype(np.float32)
+    pl[1, :5] = -np.inf
+    pl[:, 7] = -np.inf  # a row with every split empty
+    ref, ref_lse = oracle.combine(po.astype(np.float64), pl.astype(np.float64))
+    out = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((R,), dtype=torch.float32, device="cuda")
+    G.gemma_attn_combine(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda(), S, R, d, out, lse)
+    torch.cuda.synchronize()
+    got = W.bf16_bits_to_f32(host_bits(out))
+    assert_close(got, ref, "combine")
+    got_lse = lse.cpu().numpy()
+    assert got_lse[7] == -np.inf
+    np.testing.assert_allclose(got_lse[np.isfinite(ref_lse)], ref_lse[np.isfinite(ref_lse)], atol=1e-5)
