@@ -1,0 +1,488 @@
+"""Benchmark of the Gemma-4-style interleaved attention path on B200.
+
+A step is one pass of the hot path over the E2B-shaped prefill block: L = 8192 tokens,
+4 sliding-window layers (W = 512, 8/4 heads, d = 256) and 1 global layer (8/1 heads,
+d = 512, K=V, p-RoPE p = 0.25). `value` is unmasked prefill TFLOP/s of that block.
+In the same run the decode path (split-KV + combine) is timed on the long-context
+decode shape (batch 8, 32/4 heads, global K=V cache of 131072 tokens at d = 512;
+local 1024-slot ring at d = 256, 32/16 heads) and reported in HBM GB/s.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs an independent replica (weak scaling); rank 0 prints
+one JSON line with the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "prefill TFLOP/s (unmasked FLOPs) and decode HBM GB/s per layer kind, % roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def log(msg: str) -> None:
+    print(f"[bench {time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.idx)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower().startswith("active")})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+
+def sample_rows(L: int, n_rand: int, seed: int = 1):
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(128, L))) | set(range(max(0, L - 128), L))
+    rows |= set(int(x) for x in rng.integers(0, L, size=n_rand))
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+def oracle_sample_flops(layer: W.LayerSpec, rows: np.ndarray) -> int:
+    pairs = 0
+    for i in rows.tolist():
+        vis = i + 1 if layer.kind == W.GLOBAL else min(i + 1, layer.window)
+        pairs += vis
+    return 4 * layer.head_dim * layer.num_q_heads * pairs
+
+
+def cpu_baseline(wl: W.PrefillWorkload, n_rand: int = 256):
+    """Time the fp64 oracle on a bounded row sample of every layer of the block."""
+    import oracle
+    oracle.build()
+    L = wl.total_tokens
+    rows = sample_rows(L, n_rand)
+    pos = wl.positions()
+    cu = wl.cu_seqlens()
+    flops = 0
+    elapsed = 0.0
+    done = set()
+    for li, layer in enumerate(wl.layers):
+        key = (layer.kind, layer.window, layer.head_dim, layer.num_q_heads, layer.num_kv_heads)
+        q, k, v = W.layer_inputs(layer, L, wl.seed, li)
+        t0 = time.perf_counter()
+        oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                         q, k, v, pos, cu, rows=rows)
+        elapsed += time.perf_counter() - t0
+        flops += oracle_sample_flops(layer, rows)
+        done.add(key)
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} query rows (first 128, last 128, {n_rand} from default_rng(1)) x all heads "
+                      f"of each of the {len(wl.layers)} layers, fp64 C oracle with OpenMP",
+            "seconds": elapsed}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, local = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    wl = W.e2b_block()
+    L = wl.total_tokens
+    pos, cu = wl.positions(), wl.cu_seqlens()
+    inputs = [W.layer_inputs(layer, L, wl.seed, li) for li, layer in enumerate(wl.layers)]
+    rows = sample_rows(L, 0)[:64]  # a bounded sample per step (first 64 rows) keeps each step to seconds
+    rows = np.concatenate([rows, np.arange(L - 64, L, dtype=np.int32)])
+
+    def step():
+        f = 0
+        for li, layer in enumerate(wl.layers):
+            q, k, v = inputs[li]
+            oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                             q, k, v, pos, cu, rows=rows)
+            f += oracle_sample_flops(layer, rows)
+        return f
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    flops = 0
+    for _ in range(args.steps):
+        flops += step()
+    el = time.perf_counter() - t0
+    value = flops / el / 1e12
+    sample = (f"{len(rows)} query rows (first 64, last 64) x all heads of each layer of the E2B block per step, "
+              "fp64 C oracle with OpenMP")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L, "layers": "4 local (W=512) + 1 global"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import global_interleaved_layers_b200 as G
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush_buf.fill_(1.0)
+
+    # ------------------------------------------------------------------ prefill block inputs
+    wl = W.e2b_block()
+    L = wl.total_tokens
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    layers = []
+    max_ws = 0
+    for li, layer in enumerate(wl.layers):
+        q = torch.randn((L, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        k = torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        v = None if layer.k_eq_v else torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen,
+                                                 device=dev).to(torch.bfloat16)
+        out = torch.empty_like(q)
+        p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
+                     rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
+        ws_bytes = G.gemma_attn_prefill_workspace_size(p, L)
+        max_ws = max(max_ws, ws_bytes)
+        layers.append(dict(spec=layer, q=q, k=k, v=v, out=out, p=p, flops=W.prefill_flops(wl.seq_lens, layer)))
+    ws = torch.empty(max(max_ws, 256), dtype=torch.uint8, device=dev)
+    pos = torch.from_numpy(wl.positions()).to(dev)
+    cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
+    total_flops = sum(l["flops"] for l in layers)
+
+    stream = torch.cuda.current_stream()
+    kind_ev = {}  # per layer index: list of (start, end) events, recorded on the launch stream
+
+    def run_layer(li, record=False):
+        l = layers[li]
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        G.gemma_attn_prefill(l["p"], l["q"], l["k"], l["v"], l["out"], None, pos, cu, 1, L, L, ws, ws.numel(),
+                             stream)
+        n = G.gemma_attn_last_launch_count()
+        if record:
+            e1.record(stream)
+            kind_ev.setdefault(li, []).append((e0, e1))
+        return n
+
+    def step(record=False):
+        n = 0
+        for li in range(len(layers)):
+            n += run_layer(li, record)
+        return n
+
+    log("prefill warmup")
+    for _ in range(args.warmup):
+        step()
+    G.gemma_attn_check()
+    torch.cuda.synchronize()
+    log("prefill timed")
+
+    step_events = []
+    launches = 0
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            flush_l2()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            launches += step(record=True)
+            s1.record(stream)
+            step_events.append((s0, s1))
+        torch.cuda.synchronize()
+        barrier()
+    clk = clocks.summary()
+    G.gemma_attn_check()
+    step_ms = [a.elapsed_time(b) for a, b in step_events]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * total_flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    per_layer_ms = {li: float(np.mean([a.elapsed_time(b) for a, b in evs])) for li, evs in kind_ev.items()}
+    glob = [li for li, l in enumerate(layers) if l["spec"].kind == W.GLOBAL]
+    loc = [li for li, l in enumerate(layers) if l["spec"].kind == W.LOCAL]
+    g_ms = float(np.mean([per_layer_ms[i] for i in glob]))
+    l_ms = float(np.mean([per_layer_ms[i] for i in loc]))
+    g_flops = layers[glob[0]]["flops"]
+    l_flops = layers[loc[0]]["flops"]
+    g_tflops = g_flops / (g_ms * 1e-3) / 1e12
+    l_tflops = l_flops / (l_ms * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    loc_spec = layers[loc[0]]["spec"]
+    local_ceiling = loc_spec.window / (loc_spec.window + 128 - 1)
+
+    # ------------------------------------------------------------------ e2e through host buffers
+    host = []
+    h2d = d2h = 0
+    for l in layers:
+        hq = l["q"].cpu().pin_memory()
+        hk = l["k"].cpu().pin_memory()
+        hv = None if l["v"] is None else l["v"].cpu().pin_memory()
+        ho = torch.empty(l["out"].shape, dtype=torch.bfloat16).pin_memory()
+        host.append((hq, hk, hv, ho))
+        h2d += hq.numel() * 2 + hk.numel() * 2 + (0 if hv is None else hv.numel() * 2)
+        d2h += ho.numel() * 2
+
+    def e2e_step():
+        for li, l in enumerate(layers):
+            hq, hk, hv, ho = host[li]
+            l["q"].copy_(hq, non_blocking=True)
+            l["k"].copy_(hk, non_blocking=True)
+            if hv is not None:
+                l["v"].copy_(hv, non_blocking=True)
+            run_layer(li)
+            ho.copy_(l["out"], non_blocking=True)
+
+    log("e2e")
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, args.steps // 2)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
+    e2e_value = world * total_flops / (e2e_ms * 1e-3) / 1e12
+
+    # ------------------------------------------------------------------ decode (long context)
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L,
+                   "layers": "4 local (W=512, 8/4 heads, d=256) + 1 global (8/1 heads, d=512, K=V, p=0.25)",
+                   "l2": "flushed before every timed step (256 MiB write); per-step CUDA events",
+                   "parallelism": f"replicas x{world}"},
+        "per_kind": {
+            "local_prefill": {"tflops": l_tflops, "ms": l_ms, "frac_of_peak": l_tflops / peak_t,
+                              "tile_geometry_ceiling": local_ceiling},
+            "global_prefill": {"tflops": g_tflops, "ms": g_ms, "frac_of_peak": g_tflops / peak_t},
+        },
+        "roofline": {"bound": "tensor", "achieved": g_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": g_tflops / peak_t, "traffic": None,
+                     "kernel": "prefill_kernel<512> (global layer; timed call also launches the two small "
+                               "rotated-side-copy kernels)",
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if decode is not None:
+        result["per_kind"].update(decode)
+    if rank == 0 and not args.no_cpu_baseline:
+        log("cpu baseline")
+        result["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
+    wl = W.long_decode()
+    B, n_q = wl.batch, wl.n_q
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    res = {}
+    for layer in wl.layers:
+        Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+        ctx = wl.cache_lens[0]
+        if layer.kind == W.GLOBAL:
+            cap = ctx
+            layout = G.CACHE_CONTIGUOUS
+        else:
+            cap = layer.window
+            layout = G.CACHE_RING
+        kc = torch.empty((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev)
+        kc.normal_(generator=gen)
+        vc = None
+        if not layer.k_eq_v:
+            vc = torch.empty_like(kc)
+            vc.normal_(generator=gen)
+        q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+        nk = torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+        nv = None if layer.k_eq_v else torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        p = G.params(layer.kind, Hq, Hkv, d, window=layer.window, rope_p=layer.rope_p, rope_base=layer.rope_base,
+                     softmax_scale=layer.softmax_scale)
+        splits = G.gemma_attn_decode_num_splits(p, B, n_q, ctx)
+        rows = B * n_q * Hq
+        po = torch.empty((splits, rows, d), dtype=torch.float32, device=dev)
+        pl = torch.empty((splits, rows), dtype=torch.float32, device=dev)
+        out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
+
+        log(f"decode kind={layer.kind}")
+
+        def one():
+            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+
+        for _ in range(args.warmup):
+            one()
+        torch.cuda.synchronize()
+        G.gemma_attn_check()
+        evs = []
+        dec_evs = []
+        barrier()
+        for _ in range(args.steps):
+            flush_l2()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+            e1.record(stream)
+            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+            e2.record(stream)
+            evs.append((e0, e2))
+            dec_evs.append((e0, e1))
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+        dec_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dec_evs])))
+        nbytes = W.decode_cache_bytes(B, wl.cache_lens, layer)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        name = "global_decode" if layer.kind == W.GLOBAL else "local_decode"
+        res[name] = {"gbs": gbs, "ms": ms, "decode_kernel_ms": dec_ms, "bytes": nbytes, "splits": splits,
+                     "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                     "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} ctx={ctx} " + ("K=V contiguous" if layer.k_eq_v
+                                                                             else f"ring W={layer.window}")}
+        del kc, vc
+        torch.cuda.empty_cache()
+    return res
+
+
+if __name__ == "__main__":
+    main()

@@ -25,6 +25,8 @@ LOCAL = 0
 GLOBAL = 1
 CACHE_CONTIGUOUS = 0
 CACHE_RING = 1
+OUT_BF16 = 0
+OUT_F32 = 1
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -40,7 +42,8 @@ ERR_SEQLEN = -8
 class GemmaAttnParams(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("window", ctypes.c_int32), ("rope_p", ctypes.c_float),
                 ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32)]
 
 
 class GemmaAttnError(RuntimeError):
@@ -61,7 +64,7 @@ _lib.gemma_attn_prefill_workspace_size.argtypes = [_PP, _I, ctypes.POINTER(ctype
 _lib.gemma_attn_prefill.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
 _lib.gemma_attn_decode.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _I, _P]
 _lib.gemma_attn_decode_num_splits.argtypes = [_PP, _I, _I, _I, ctypes.POINTER(ctypes.c_int32)]
-_lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
+_lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_tile_plan.argtypes = [_I, _I, _P, _I, _I, _I, _P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
 _lib.gemma_attn_check.argtypes = [_P]
 _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
@@ -72,10 +75,12 @@ for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_att
 
 
 def params(kind: int, num_q_heads: int, num_kv_heads: int, head_dim: int, window: int = 0,
-           rope_p: float = 1.0, rope_base: float = 10000.0, softmax_scale: Optional[float] = None) -> GemmaAttnParams:
+           rope_p: float = 1.0, rope_base: float = 10000.0, softmax_scale: Optional[float] = None,
+           out_dtype: int = OUT_BF16) -> GemmaAttnParams:
     if softmax_scale is None:
         softmax_scale = head_dim ** -0.5
-    return GemmaAttnParams(kind, window, rope_p, rope_base, softmax_scale, num_q_heads, num_kv_heads, head_dim)
+    return GemmaAttnParams(kind, window, rope_p, rope_base, softmax_scale, num_q_heads, num_kv_heads, head_dim,
+                           out_dtype)
 
 
 def _ptr(x) -> Optional[int]:
@@ -145,10 +150,10 @@ def gemma_attn_decode_num_splits(p: GemmaAttnParams, batch: int, n_q: int, max_c
     return int(n.value)
 
 
-def gemma_attn_combine(partial_o, partial_lse, num_splits: int, rows: int, head_dim: int, out, lse,
-                       stream=None) -> None:
-    _check(_lib.gemma_attn_combine(_ptr(partial_o), _ptr(partial_lse), num_splits, rows, head_dim, _ptr(out),
-                                   _ptr(lse), _stream(stream)), "gemma_attn_combine")
+def gemma_attn_combine(partial_o, partial_lse, num_splits: int, rows: int, head_dim: int, out_dtype: int, out,
+                       lse, stream=None) -> None:
+    _check(_lib.gemma_attn_combine(_ptr(partial_o), _ptr(partial_lse), num_splits, rows, head_dim, out_dtype,
+                                   _ptr(out), _ptr(lse), _stream(stream)), "gemma_attn_combine")
 
 
 def gemma_attn_tile_plan(kind: int, window: int, cu_seqlens_host, bm: int, bn: int):

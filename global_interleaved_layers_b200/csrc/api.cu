@@ -65,6 +65,7 @@ int check_params(const gemma_attn_params* p) {
   if (p->kind == GEMMA_ATTN_LOCAL && p->window < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (!(p->rope_p >= 0.f && p->rope_p <= 1.f)) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (!(p->rope_base > 0.f) || !(p->softmax_scale > 0.f)) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (p->out_dtype != GEMMA_ATTN_OUT_BF16 && p->out_dtype != GEMMA_ATTN_OUT_F32) return GEMMA_ATTN_ERR_INVALID_ARG;
   return GEMMA_ATTN_OK;
 }
 
@@ -208,6 +209,7 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
   a.max_qtiles = (max_seqlen + 127) / 128; a.max_seqlen = max_seqlen; a.total_tokens = total_tokens;
   a.num_q_heads = Hq; a.group = Hq / Hkv; a.head_dim = d; a.is_local = global ? 0 : 1;
   a.window = global ? 0 : params->window; a.softmax_scale = params->softmax_scale; a.rot_mask = L.mask;
+  a.out_f32 = params->out_dtype == GEMMA_ATTN_OUT_F32;
   cudaError_t e;
   switch (L.kd) {
     case 64: e = launch_prefill<64>(maps, a, stream); break;
@@ -275,13 +277,15 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
 }
 
 int gemma_attn_combine(const float* partial_o, const float* partial_lse, int32_t num_splits, int32_t rows,
-                       int32_t head_dim, void* out, float* lse, void* stream_) {
+                       int32_t head_dim, int32_t out_dtype, void* out, float* lse, void* stream_) {
   t_launches = 0;
   if (!partial_o || !partial_lse || !out || num_splits < 1 || rows < 0 || head_dim < 1)
     return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (out_dtype != GEMMA_ATTN_OUT_BF16 && out_dtype != GEMMA_ATTN_OUT_F32) return GEMMA_ATTN_ERR_INVALID_ARG;
   CombineArgs a;
   a.partial_o = partial_o; a.partial_lse = partial_lse; a.out = out; a.lse = lse;
   a.num_splits = num_splits; a.rows = rows; a.head_dim = head_dim;
+  a.out_f32 = out_dtype == GEMMA_ATTN_OUT_F32;
   if (launch_combine(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
   t_launches = rows > 0 ? 1 : 0;
   return GEMMA_ATTN_OK;

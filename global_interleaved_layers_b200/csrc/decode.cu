@@ -245,7 +245,6 @@ __global__ void combine_kernel(CombineArgs a) {
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.head_dim;
   for (int c = lane; c < a.head_dim; c += 32) {
     float acc = 0.f;
     if (mm != -INFINITY) {
@@ -256,7 +255,10 @@ __global__ void combine_kernel(CombineArgs a) {
       }
       acc /= den;
     }
-    out[c] = __float2bfloat16_rn(acc);
+    if (a.out_f32)
+      reinterpret_cast<float*>(a.out)[(size_t)row * a.head_dim + c] = acc;
+    else
+      reinterpret_cast<__nv_bfloat16*>(a.out)[(size_t)row * a.head_dim + c] = __float2bfloat16_rn(acc);
   }
   if (lane == 0 && a.lse != nullptr) a.lse[row] = (mm == -INFINITY) ? -INFINITY : mm + logf(den);
 }

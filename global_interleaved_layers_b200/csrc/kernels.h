@@ -21,6 +21,7 @@ struct PrefillArgs {
   int is_local;
   int window;
   float softmax_scale;
+  int out_f32;        // 1: write fp32 output, 0: bf16
   uint32_t rot_mask;  // bit c set: key/query chunk c (64 dims) is read from the rotated side copy
 };
 
@@ -69,6 +70,7 @@ struct CombineArgs {
   void* out;
   float* lse;
   int num_splits, rows, head_dim;
+  int out_f32;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 

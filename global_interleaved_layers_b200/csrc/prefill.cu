@@ -168,11 +168,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         }
       }
       // Let every copy this thread issued land before the CTA can exit: the last
-      // kStages loads are the only ones that may still be in flight.
+      // kStages loads are the only ones that may still be in flight. (st, ph) is the
+      // next slot to fill; each slot's most recent fill completed the phase of parity
+      // ph ^ 1 (the wrap inside next() flips ph for the slots filled this round).
       for (int s = 0; s < Cfg::kStages; ++s) {
-        if (!mbar_try_wait(&bars->ring_full[st], ph)) {
+        if (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u)) {
           unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&bars->ring_full[st], ph) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+          while (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {}
         }
         next();
         (void)s;
@@ -260,7 +262,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       for (int c = 0; c < kBN / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
       tmem_ld_wait();
       const int kt = kt_lo + jj;
-      const bool partial = kv_tile_class(is_local, args.window, len, qt, kt, kBM, kBN) != kTileFull;
+      // A key tile that runs past the end of the sequence holds the next sequence's
+      // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
+      const bool partial = (kt + 1) * kBN > len ||
+                           kv_tile_class(is_local, args.window, len, qt, kt, kBM, kBN) != kTileFull;
       float m_tile = -INFINITY;
       if (partial) {
         const int k0 = kt * kBN;
@@ -324,21 +329,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
       const bool valid = grow < len;
       const int tok = tok0 + grow;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) +
-                            ((size_t)tok * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv;
+      const size_t obase = ((size_t)tok * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv;
 #pragma unroll 1
       for (int c = 0; c < Cfg::kDv / 32; ++c) {
         uint32_t o[32];
         tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
         tmem_ld_wait();
         if (valid && vpart * Cfg::kDv + c * 32 < args.head_dim) {
-          uint32_t w[16];
+          if (args.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out) + obase + c * 32);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                   __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+          } else {
+            uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.out) + obase + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
         }
       }
       if (valid && vpart == 0 && args.lse != nullptr)

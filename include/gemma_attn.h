@@ -68,9 +68,15 @@ enum {
   GEMMA_ATTN_ERR_SEQLEN = -8
 };
 
+enum {
+  GEMMA_ATTN_OUT_BF16 = 0, /* outputs rounded to bfloat16 (round to nearest even) */
+  GEMMA_ATTN_OUT_F32 = 1   /* outputs left in the fp32 accumulator precision */
+};
+
 /* Layer description. head_dim in {32, 64, 128, 256, 512}; num_q_heads a multiple of
  * num_kv_heads; window >= 1 for LOCAL (ignored for GLOBAL); 0 <= rope_p <= 1;
- * rope_base > 0; softmax_scale > 0 (typically 1/sqrt(head_dim)). */
+ * rope_base > 0; softmax_scale > 0 (typically 1/sqrt(head_dim)); out_dtype selects
+ * the element type of `out` (GEMMA_ATTN_OUT_BF16 or GEMMA_ATTN_OUT_F32). */
 typedef struct gemma_attn_params {
   int32_t kind;
   int32_t window;
@@ -80,6 +86,7 @@ typedef struct gemma_attn_params {
   int32_t num_q_heads;
   int32_t num_kv_heads;
   int32_t head_dim;
+  int32_t out_dtype;
 } gemma_attn_params;
 
 /* Bytes of device workspace gemma_attn_prefill needs for `total_tokens` tokens
@@ -95,7 +102,7 @@ int gemma_attn_prefill_workspace_size(const gemma_attn_params* params, int32_t t
  *   q         [total_tokens, num_q_heads, head_dim] bf16, device.
  *   k         [total_tokens, num_kv_heads, head_dim] bf16, device (GLOBAL: the K=V tensor).
  *   v         same shape as k for LOCAL; must be NULL for GLOBAL (values = k, un-rotated).
- *   out       [total_tokens, num_q_heads, head_dim] bf16, device, written.
+ *   out       [total_tokens, num_q_heads, head_dim] bf16 or f32 (params->out_dtype), device, written.
  *   lse       [num_q_heads, total_tokens] float32 natural-log sum-exp of the scaled
  *             scores, device, written; may be NULL.
  *   positions [total_tokens] int32, device: rotary position of each token. Within a
@@ -148,10 +155,11 @@ int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch,
  * Combine split partials: out = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M) with
  * M = max_s lse_s; lse = M + log(sum_s exp(lse_s - M)).
  *   partial_o [num_splits, rows, head_dim] f32, partial_lse [num_splits, rows] f32 (device).
- *   out [rows, head_dim] bf16 (device, written); lse [rows] f32 or NULL.
+ *   out [rows, head_dim] (device, written): bf16 or f32 per out_dtype; lse [rows] f32 or NULL.
  */
 int gemma_attn_combine(const float* partial_o, const float* partial_lse, int32_t num_splits,
-                       int32_t rows, int32_t head_dim, void* out, float* lse, void* stream);
+                       int32_t rows, int32_t head_dim, int32_t out_dtype, void* out, float* lse,
+                       void* stream);
 
 /*
  * Host-side tile plan (the same rule the prefill kernels apply): for every sequence,

@@ -46,8 +46,15 @@ def assert_close(got, ref, what=""):
     return max_abs, rel_rms
 
 
-def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=True):
-    """q/k/v: bf16 bit arrays (host) or bf16 device tensors. Returns (out bf16 device, lse device)."""
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 (round to nearest even) -> float32."""
+    return W.bf16_bits_to_f32(W.f32_to_bf16_bits(np.asarray(x, dtype=np.float32)))
+
+
+def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=True, out_f32=False):
+    """q/k/v: bf16 bit arrays (host) or bf16 device tensors. Returns (out device tensor, lse device).
+
+    out is bf16 unless out_f32 (then float32, the accumulator precision)."""
     qd = q if isinstance(q, torch.Tensor) else dev_bf16(q)
     kd = k if isinstance(k, torch.Tensor) else dev_bf16(k)
     vd = None if v is None else (v if isinstance(v, torch.Tensor) else dev_bf16(v))
@@ -56,8 +63,9 @@ def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=
     S = cu.shape[0] - 1
     max_len = int(np.max(np.diff(cu)))
     p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
-                 rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
-    out = torch.empty_like(qd)
+                 rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale,
+                 out_dtype=G.OUT_F32 if out_f32 else G.OUT_BF16)
+    out = torch.empty(qd.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
     lse = torch.empty((Hq, T), dtype=torch.float32, device="cuda") if with_lse else None
     ws_bytes = G.gemma_attn_prefill_workspace_size(p, T)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")

@@ -1,7 +1,9 @@
 """GPU parity: the CUDA path (called through the C-ABI) against the fp64 oracle.
 
-Bounds (from the acceptance criteria): max-abs <= 1e-2 and relative RMS <= 5e-3 on
-outputs; lse within 1e-2. Shapes span several 128-row tiles with ragged tails, GQA
+Bounds (from the acceptance criteria, bf16 in, fp32 accumulate): max-abs <= 1e-2 and
+relative RMS <= 5e-3 on the fp32 outputs; lse within 1e-2. The bf16 output mode must
+equal the fp32 output rounded to nearest even, bit for bit (a bf16 half-ulp alone is
+1.6e-2 for |o| in [4, 8), so the bound is applied before that final rounding). Shapes span several 128-row tiles with ragged tails, GQA
 ratios 2:1 and 8:1, head dims 32..512, windows from 1 to beyond the length,
 K=V with p-RoPE, and position offsets.
 """
@@ -17,7 +19,8 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 G = pytest.importorskip("global_interleaved_layers_b200")
-from gpu_util import assert_close, dev_bf16, dev_i32, host_bits, ring_from_history, run_prefill  # noqa: E402
+from gpu_util import (assert_close, bf16_round, dev_bf16, dev_i32, host_bits, ring_from_history,  # noqa: E402
+                      run_prefill)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -62,9 +65,11 @@ def _check_prefill(layer, seq_lens, seed=0, pos_start=0, rows=None):
     q, k, v = W.layer_inputs(layer, T, seed)
     cu = np.concatenate([[0], np.cumsum(seq_lens)]).astype(np.int32)
     pos = np.concatenate([np.arange(n) + pos_start for n in seq_lens]).astype(np.int32)
-    out, lse = run_prefill(G, layer, q, k, v, pos, cu)
-    got = W.bf16_bits_to_f32(host_bits(out))
+    out32, lse = run_prefill(G, layer, q, k, v, pos, cu, out_f32=True)
+    out16, _ = run_prefill(G, layer, q, k, v, pos, cu, with_lse=False)
+    got = out32.cpu().numpy()
     got_lse = lse.cpu().numpy()
+    np.testing.assert_array_equal(W.bf16_bits_to_f32(host_bits(out16)), bf16_round(got))
     ref, ref_lse = oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
                                     q, k, v, pos, cu, rows=rows)
     if rows is not None:
@@ -158,11 +163,14 @@ def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11):
     G.gemma_attn_decode(p, dev_bf16(q), dev_bf16(new_k), None if new_v is None else dev_bf16(new_v), dev_bf16(kc),
                         None if vc is None else dev_bf16(vc), layout, cap, dev_i32(cache_lens), B, n_q, max_len,
                         po, pl, num_splits)
-    out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((B, n_q, Hq, d), dtype=torch.float32, device="cuda")
+    out16 = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
-    G.gemma_attn_combine(po, pl, num_splits, rows, d, out, lse)
+    G.gemma_attn_combine(po, pl, num_splits, rows, d, G.OUT_F32, out, lse)
+    G.gemma_attn_combine(po, pl, num_splits, rows, d, G.OUT_BF16, out16, None)
     G.gemma_attn_check()
-    got = W.bf16_bits_to_f32(host_bits(out))
+    got = out.cpu().numpy()
+    np.testing.assert_array_equal(W.bf16_bits_to_f32(host_bits(out16)), bf16_round(got))
     assert_close(got, ref, f"decode {layer} lens={cache_lens} n_q={n_q} splits={num_splits}")
     np.testing.assert_allclose(lse.cpu().numpy().reshape(ref_lse.shape), ref_lse, atol=1e-2, rtol=0)
 
@@ -206,11 +214,11 @@ def test_combine_against_oracle():
     pl[1, :5] = -np.inf
     pl[:, 7] = -np.inf  # a row with every split empty
     ref, ref_lse = oracle.combine(po.astype(np.float64), pl.astype(np.float64))
-    out = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((R, d), dtype=torch.float32, device="cuda")
     lse = torch.empty((R,), dtype=torch.float32, device="cuda")
-    G.gemma_attn_combine(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda(), S, R, d, out, lse)
+    G.gemma_attn_combine(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda(), S, R, d, G.OUT_F32, out, lse)
     torch.cuda.synchronize()
-    got = W.bf16_bits_to_f32(host_bits(out))
+    got = out.cpu().numpy()
     assert_close(got, ref, "combine")
     got_lse = lse.cpu().numpy()
     assert got_lse[7] == -np.inf
