@@ -253,7 +253,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     for (int jj = 0; jj < ntiles && ok; ++jj) {
       const int b = jj & 1;
       const uint32_t s_col = b ? kColS1 : kColS0;
-      ok = mbar_wait(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float t[kBN];
@@ -285,26 +285,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       }
       // O may only be touched once PV(jj-1) has finished.
       if (jj >= 1) {
-        ok = mbar_wait(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag));
         if (!ok) break;
         tc_fence_after();
       }
+      // Raise the running max only when it grows by more than 2^8 (or was empty); P
+      // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
+      float alpha = 1.f;
+      bool rescale_o = false;
       if (m_tile > m_used + kRescaleThreshold || (m_used == -INFINITY && m_tile > -INFINITY)) {
         if (m_used != -INFINITY) {
-          const float alpha = fast_exp2(m_used - m_tile);
+          alpha = fast_exp2(m_used - m_tile);
           l_sum *= alpha;
-          // rescale this row of O (written by PV(0..jj-1))
-#pragma unroll 1
-          for (int c = 0; c < Cfg::kDv / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
-          }
+          rescale_o = true;
         }
         m_used = m_tile;
+      }
+      // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
+      // lane needs it, each lane with its own factor (1 for lanes that do not).
+      if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll 1
+        for (int c = 0; c < Cfg::kDv / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
+        }
       }
       const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t p[kBN / 2];
@@ -323,7 +331,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       tc_fence_before();
       mbar_arrive(&bars->p_full[b]);
     }
-    if (ok && ntiles > 0) ok = mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag);
+    if (ok && ntiles > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag));
     if (ok) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -361,6 +370,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    // tcgen05.dealloc is warp-collective: lane 0 ran the MMA loop alone, so the warp
+    // reconverges explicitly before the whole warp frees the columns.
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

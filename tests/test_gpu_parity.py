@@ -223,3 +223,23 @@ def test_combine_against_oracle():
     got_lse = lse.cpu().numpy()
     assert got_lse[7] == -np.inf
     np.testing.assert_allclose(got_lse[np.isfinite(ref_lse)], ref_lse[np.isfinite(ref_lse)], atol=1e-5)
+
+
+def test_prefill_divergent_rescale_within_warp():
+    """One key with a huge score: rows at or after it raise their running max by far more
+    than 2^8 mid-sequence, rows before it do not, so lanes of one warp disagree."""
+    T, d = 400, 64
+    layer = W.LayerSpec(W.GLOBAL, 2, 1, d, rope_p=0.0, rope_base=1e4)
+    rng = np.random.default_rng(31)
+    qf = np.zeros((T, 2, d), np.float32)
+    qf[:, :, 0] = 4.0
+    kf = (rng.standard_normal((T, 1, d)) * 0.1).astype(np.float32)
+    kf[300, 0, 0] = 40.0
+    q = W.f32_to_bf16_bits(qf)
+    k = W.f32_to_bf16_bits(kf)
+    pos = np.arange(T, dtype=np.int32)
+    cu = np.array([0, T], np.int32)
+    out, lse = run_prefill(G, layer, q, k, None, pos, cu, out_f32=True)
+    ref, ref_lse = oracle.attention(layer.kind, 0, 0.0, 1e4, layer.softmax_scale, q, k, None, pos, cu)
+    assert_close(out.cpu().numpy(), ref, "divergent rescale")
+    np.testing.assert_allclose(lse.cpu().numpy().T, ref_lse, atol=1e-2, rtol=0)
