@@ -209,11 +209,19 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--case", default="block",
+                    choices=["block", "global_prefill", "local_prefill", "global_decode", "local_decode"],
+                    help="block: the benchmark (one JSON line). Any other value runs only that operation "
+                         "(warmup + steps launches, no timing contract) for profiler captures.")
+    ap.add_argument("--ctx", type=int, default=0, help="decode cases: cached tokens per sequence (0: 131072)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.case != "block":
+        run_case(args)
         return
 
     import torch
@@ -482,6 +490,63 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
         del kc, vc
         torch.cuda.empty_cache()
     return res
+
+
+def run_case(args):
+    """One operation of the hot path on its benchmark shape, for profiler captures."""
+    import torch
+    import global_interleaved_layers_b200 as G
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    if args.case.endswith("prefill"):
+        wl = W.e2b_block()
+        layer = wl.layers[-1] if args.case == "global_prefill" else wl.layers[0]
+        L = wl.total_tokens
+        q = torch.randn((L, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        k = torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        v = None if layer.k_eq_v else torch.randn_like(k)
+        out = torch.empty_like(q)
+        p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
+                     rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
+        ws_bytes = G.gemma_attn_prefill_workspace_size(p, L)
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        pos = torch.from_numpy(wl.positions()).to(dev)
+        cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
+
+        def op():
+            G.gemma_attn_prefill(p, q, k, v, out, None, pos, cu, 1, L, L, ws, ws_bytes, stream)
+    else:
+        wl = W.long_decode()
+        layer = wl.layers[0] if args.case == "global_decode" else wl.layers[1]
+        B, n_q, ctx = wl.batch, wl.n_q, (args.ctx or wl.cache_lens[0])
+        Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+        cap = ctx if layer.k_eq_v else layer.window
+        layout = G.CACHE_CONTIGUOUS if layer.k_eq_v else G.CACHE_RING
+        kc = torch.empty((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev).normal_(generator=gen)
+        vc = None if layer.k_eq_v else torch.empty_like(kc).normal_(generator=gen)
+        q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+        nk = torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+        nv = None if layer.k_eq_v else torch.randn_like(nk)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        p = G.params(layer.kind, Hq, Hkv, d, window=layer.window, rope_p=layer.rope_p, rope_base=layer.rope_base,
+                     softmax_scale=layer.softmax_scale)
+        splits = G.gemma_attn_decode_num_splits(p, B, n_q, ctx)
+        rows = B * n_q * Hq
+        po = torch.empty((splits, rows, d), dtype=torch.float32, device=dev)
+        pl = torch.empty((splits, rows), dtype=torch.float32, device=dev)
+        out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
+
+        def op():
+            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+    for _ in range(args.warmup + args.steps):
+        op()
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    print(json.dumps({"case": args.case, "launches": args.warmup + args.steps}), flush=True)
 
 
 if __name__ == "__main__":
