@@ -66,11 +66,12 @@ _lib.gemma_attn_decode.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, 
 _lib.gemma_attn_decode_num_splits.argtypes = [_PP, _I, _I, _I, ctypes.POINTER(ctypes.c_int32)]
 _lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_tile_plan.argtypes = [_I, _I, _P, _I, _I, _I, _P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+_lib.gemma_attn_decode_noalloc.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_check.argtypes = [_P]
 _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
 for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_attn_decode",
            "gemma_attn_decode_num_splits", "gemma_attn_combine", "gemma_attn_tile_plan", "gemma_attn_check",
-           "gemma_attn_selftest_umma"):
+           "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -141,6 +142,19 @@ def gemma_attn_decode(p: GemmaAttnParams, q, new_k, new_v, k_cache, v_cache, cac
                                   _ptr(v_cache), cache_layout, cache_capacity, _ptr(cache_seqlens), batch, n_q,
                                   max_cache_len, _ptr(partial_o), _ptr(partial_lse), num_splits, _stream(stream)),
            "gemma_attn_decode")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def gemma_attn_decode_noalloc(p: GemmaAttnParams, q, new_k, new_v, k_cache, v_cache, cache_layout: int,
+                              cache_capacity: int, cache_seqlens, batch: int, n_q: int, max_cache_len: int,
+                              num_splits: int, out, lse, stream=None) -> None:
+    """Decode + combine with the split partials in the library's static device array (no allocation)."""
+    _check(_lib.gemma_attn_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(new_k), _ptr(new_v), _ptr(k_cache),
+                                          _ptr(v_cache), cache_layout, cache_capacity, _ptr(cache_seqlens), batch,
+                                          n_q, max_cache_len, num_splits, _ptr(out), _ptr(lse), _stream(stream)),
+           "gemma_attn_decode_noalloc")
 
 
 def gemma_attn_decode_num_splits(p: GemmaAttnParams, batch: int, n_q: int, max_cache_len: int) -> int:

@@ -4,4 +4,5 @@
 #include "rope.cu"
 #include "prefill.cu"
 #include "decode.cu"
+#include "decode_noalloc.cu"
 #include "selftest.cu"

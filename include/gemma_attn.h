@@ -147,6 +147,38 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
                       int32_t batch, int32_t n_q, int32_t max_cache_len,
                       float* partial_o, float* partial_lse, int32_t num_splits, void* stream);
 
+/*
+ * Decode + combine in one call that allocates nothing. The pages have no counterpart
+ * to this entry point: it serves callers of this library that cannot allocate device
+ * memory -- an op inside a framework that owns every device allocation and offers it
+ * no scratch allocator, or a caller capturing a CUDA graph, where cudaMalloc is not
+ * allowed -- so they cannot provide the split partials that gemma_attn_decode writes.
+ * Here the partials live in a static array of GEMMA_ATTN_NOALLOC_SCRATCH_BYTES inside
+ * the library; every GPU that loads the library holds it until the process exits.
+ *   Arguments: as gemma_attn_decode (q, new_k, new_v, caches, layout, capacity,
+ *   cache_seqlens, batch, n_q, max_cache_len, num_splits), then out [batch, n_q,
+ *   num_q_heads, head_dim] (bf16 or f32 per params->out_dtype) and lse [batch * n_q *
+ *   num_q_heads] f32 or NULL, as gemma_attn_combine writes them. The caller passes and
+ *   owns every input and output buffer.
+ *   Limit: num_splits * batch * n_q * num_q_heads * (head_dim + 1) * 4 bytes (each of
+ *   the two partial arrays rounded up to 256 bytes) must not exceed
+ *   GEMMA_ATTN_NOALLOC_SCRATCH_BYTES; a larger request returns GEMMA_ATTN_ERR_WORKSPACE
+ *   and launches nothing (use fewer splits).
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any
+ *   stream capture. All calls share the array and it keeps the last call's contents;
+ *   each call rewrites every partial it reads, so nothing is cleared between calls.
+ *   Calls that overlap on the GPU (concurrent streams, or threads whose streams are
+ *   not ordered) race on the array and corrupt each other's results.
+ */
+#define GEMMA_ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+int gemma_attn_decode_noalloc(const gemma_attn_params* params, const void* q, const void* new_k,
+                              const void* new_v, const void* k_cache, const void* v_cache,
+                              int32_t cache_layout, int32_t cache_capacity,
+                              const int32_t* cache_seqlens, int32_t batch, int32_t n_q,
+                              int32_t max_cache_len, int32_t num_splits, void* out, float* lse,
+                              void* stream);
+
 /* A split count for gemma_attn_decode that fills the GPU for this shape. */
 int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,
                                  int32_t max_cache_len, int32_t* num_splits);
