@@ -230,10 +230,22 @@ int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch,
   if (batch < 1 || n_q < 1 || max_cache_len < 0 || !num_splits) return GEMMA_ATTN_ERR_INVALID_ARG;
   int keys = params->kind == GEMMA_ATTN_LOCAL ? std::min(max_cache_len, params->window) : max_cache_len;
   keys += n_q;
+  // One decode CTA per SM at a time: pick the split count whose CTA total fills whole
+  // waves of 148 best, with at least two waves' worth of CTAs where the keys allow and
+  // at least 512 keys (8 chunks) per split.
+  const int sms = 148;
   const int units = batch * params->num_kv_heads;
-  int s = (2 * 148 + units - 1) / units;              // about two CTAs per SM
-  s = std::min(s, std::max(1, keys / 64));             // at least 64 keys per split
-  *num_splits = std::max(1, s);
+  const int s_cap = std::max(1, keys / 512);
+  const int s_min = std::min(s_cap, std::max(1, (2 * sms + units - 1) / units));
+  int best = s_min;
+  double best_eff = 0.0;
+  for (int s = s_min; s <= std::min(s_cap, 4 * s_min); ++s) {
+    const long long ctas = (long long)units * s;
+    const long long waves = (ctas + sms - 1) / sms;
+    const double eff = (double)ctas / (double)(waves * sms);
+    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+  }
+  *num_splits = best;
   return GEMMA_ATTN_OK;
 }
 
@@ -256,7 +268,9 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
     return GEMMA_ATTN_ERR_INVALID_ARG;
   if (cache_capacity < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
   const int group = params->num_q_heads / params->num_kv_heads;
-  if ((group * n_q + 7) / 8 > 8) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  if (group * n_q > decode_max_rows(params->head_dim)) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
+    return GEMMA_ATTN_ERR_MISALIGNED;
   DecodeArgs a;
   a.q = static_cast<const uint16_t*>(q);
   a.new_k = static_cast<const uint16_t*>(new_k);

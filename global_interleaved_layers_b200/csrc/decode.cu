@@ -4,219 +4,493 @@
 // new tokens themselves. Local layers read a window-slot ring (token p in slot
 // p mod W); global layers read a contiguous cache holding the single K=V tensor
 // ("Visual guide to Gemma 4", sections "K=V technique" and "GQA": the KV cache is
-// what GQA and K=V shrink). Keys are stored un-rotated: the copy used for scores
-// is rotated on load (p-RoPE: only the first r pairs), values are used as loaded.
+// what GQA and K=V shrink). Keys are stored un-rotated; the copy used for scores is
+// rotated after it lands in shared memory (p-RoPE: only the first r pairs), values
+// are used as loaded.
 //
-// The visible keys of a sequence, ordered by position, are cut into `num_splits`
-// contiguous ranges; one CTA handles (sequence, KV head, split) for all query
-// heads of that KV head and all n_q tokens, and writes an unnormalised partial
-// (O / l and the log-sum-exp) that the combine kernel merges.
+// The visible keys of a sequence, in position order (cached tokens, then the new
+// tokens), are cut into `num_splits` contiguous ranges. One CTA (4 warps) handles a
+// (sequence, KV head, split) for every query head of that KV head and every new token
+// -- the "rows". Per chunk of 64 keys:
+//   1. cp.async brings the chunk's key (and, for local layers, value) rows into padded
+//      shared memory, double-buffered so the next chunk streams in meanwhile;
+//   2. the rotated copy for scores is formed (a per-thread angle recurrence over the
+//      chunk's consecutive positions, re-anchored exactly every chunk);
+//   3. S^T = K Q^T on tensor cores (mma.sync m16n8k16 bf16, keys on M, rows on N);
+//   4. online softmax per row across the 4 warps;
+//   5. O^T += V^T P^T on tensor cores, the warps splitting the head dim.
+// The CTA writes an fp32 partial (O / l) and its log-sum-exp for the combine.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace gattn {
 
 namespace {
-constexpr int kDecThreads = 256;
-constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kRowsPerWarp = 8;
+
+constexpr int kDecThreads = 128;
+constexpr int kDecWarps = 4;
+constexpr int kCK = 64;  // keys per chunk
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // 0: zero-fill, nothing read
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// D(16x8 f32) += A(16x16 bf16, row) * B(16x8 bf16, col)
+__device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Each warp owns up to 8 query rows (a row = one query head for one new token) and
-// a strided subset of the split's keys. A lane holds H = D/64 consecutive dims from
-// each half of the head (dims lane*H.. and D/2 + lane*H..), so both members of every
-// rotary pair sit in the same lane.
-template <int D>
-__global__ void __launch_bounds__(kDecThreads)
-decode_kernel(DecodeArgs a) {
-  constexpr int HALF = D / 2;
-  constexpr int H = (HALF >= 32) ? HALF / 32 : 1;   // dims per half per lane
-  constexpr int ACTIVE = (HALF >= 32) ? 32 : HALF;  // lanes holding dims
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int group = a.num_q_heads / a.num_kv_heads;
-  const int G = group * a.n_q;                       // query rows of this CTA
-  const int nrg = (G + kRowsPerWarp - 1) / kRowsPerWarp;
-  const int streams = kDecWarps / nrg;               // warps per row group (>= 1)
-  const int rg = warp % nrg;
-  const int stream_id = warp / nrg;
-  const bool warp_active = warp < nrg * streams;
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
 
+// Shared-memory carve-up of the decode kernel (element counts are bf16 unless noted).
+template <int D, int NT>
+struct DecSmem {
+  static constexpr int kRowPad = 8;                    // 16 bytes: conflict-free ldmatrix rows
+  static constexpr int KST = D + kRowPad;              // key/value/query row stride
+  static constexpr int RPAD = 8 * NT;                  // query rows, padded to n-tiles
+  static constexpr int PST = kCK + kRowPad;            // P row stride
+  static constexpr int NKS = D / 16;                   // k-steps of the head dim
+};
+
+}  // namespace
+
+// Bytes of dynamic shared memory for decode_tc_kernel<D, NT> given the rotated k-step
+// count nrk (0 when the keys are rotated in place).
+template <int D, int NT>
+__host__ __device__ constexpr size_t dec_smem_bytes(bool separate_v, int nrk) {
+  using S = DecSmem<D, NT>;
+  size_t b = 0;
+  b += 2ull * kCK * S::KST * 2;                        // key buffers
+  if (separate_v) b += 2ull * kCK * S::KST * 2;        // value buffers
+  b += (size_t)kCK * (nrk * 16 + S::kRowPad) * 2;      // rotated copy (K=V layers)
+  b += (size_t)S::RPAD * S::KST * 2;                   // rotated queries
+  b += (size_t)S::RPAD * S::PST * 2;                   // P
+  b += 2ull * kDecWarps * S::RPAD * 4;                 // per-warp row max / sum
+  b += (size_t)S::NKS * 4;                             // k-step -> rotated slot
+  return b;
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kDecThreads)
+decode_tc_kernel(DecodeArgs a) {
+  using S = DecSmem<D, NT>;
+  constexpr int HALF = D / 2;
+  constexpr int KST = S::KST;
+  constexpr int RPAD = S::RPAD;
+  constexpr int PST = S::PST;
+  constexpr int NKS = S::NKS;
+  constexpr int MT_TOTAL = D / 16;                              // 16-dim m-tiles of O^T
+  constexpr int PV_WARPS = MT_TOTAL < kDecWarps ? MT_TOTAL : kDecWarps;
+  constexpr int MTW = MT_TOTAL / PV_WARPS;                      // m-tiles per PV warp
+  constexpr int PIECES = D / 8;                                 // 16-byte pieces per row
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int group = a.num_q_heads / a.num_kv_heads;
+  const int R = group * a.n_q;
+  const bool kv_same = a.v_cache == nullptr;
   const int len = a.cache_seqlens[b];
   const int first = a.is_local ? max(0, len - a.window + 1) : 0;  // oldest position any query sees
   const int nk = (len - first) + a.n_q;
   const int per = (nk + a.num_splits - 1) / a.num_splits;
-  const int v_lo = split * per;
+  const int v_lo = min(nk, split * per);
   const int v_hi = min(nk, v_lo + per);
+  const int r = a.r;
+  // rotated k-steps (only for K=V layers, where the values must stay un-rotated)
+  int nrk = 0;
+  if (kv_same)
+    for (int s = 0; s < NKS; ++s)
+      if (s * 16 < r || (s * 16 < HALF + r && s * 16 + 16 > HALF)) ++nrk;
+  const int RST = nrk * 16 + S::kRowPad;
 
-  extern __shared__ float dsm[];
-  float* qs = dsm;                                   // [G][D] rotated, scaled queries
-  float* red = qs + (size_t)G * D;                   // [warps][8][D + 2] partial states
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint16_t* kbuf = reinterpret_cast<uint16_t*>(dsm);
+  uint16_t* vbuf = kbuf + 2 * kCK * KST;
+  uint16_t* rbuf = kv_same ? vbuf : vbuf + 2 * kCK * KST;
+  uint16_t* qs = rbuf + kCK * RST;
+  uint16_t* ps = qs + RPAD * KST;
+  float* red_max = reinterpret_cast<float*>(ps + RPAD * PST);
+  float* red_sum = red_max + kDecWarps * RPAD;
+  int* ks_slot = reinterpret_cast<int*>(red_sum + kDecWarps * RPAD);
+
+  if (tid < NKS) {
+    int slot = -1;
+    if (kv_same) {
+      int c = 0;
+      for (int s = 0; s <= tid; ++s) {
+        const bool rot = s * 16 < r || (s * 16 < HALF + r && s * 16 + 16 > HALF);
+        if (s == tid && rot) slot = c;
+        if (rot) ++c;
+      }
+    }
+    ks_slot[tid] = slot;
+  }
+
+  // ---- rotated queries (bf16) into shared memory; padding rows are zero
+  for (int idx = tid; idx < RPAD * HALF; idx += kDecThreads) {
+    const int row = idx / HALF, j = idx % HALF;
+    float y0 = 0.f, y1 = 0.f;
+    if (row < R) {
+      const int i = row / group, hh = row % group;
+      const uint16_t* qrow = a.q + (((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh) * D;
+      const float x0 = bf2f(qrow[j]), x1 = bf2f(qrow[j + HALF]);
+      y0 = x0; y1 = x1;
+      if (j < r) {
+        float c, s;
+        rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
+        y0 = x0 * c - x1 * s;
+        y1 = x0 * s + x1 * c;
+      }
+    }
+    qs[row * KST + j] = f2bf(y0);
+    qs[row * KST + j + HALF] = f2bf(y1);
+  }
+
+  // ---- rotation work assignment: thread -> pair j, walking keys ks0, ks0 + kstride, ...
+  int rj = -1, rks0 = 0, rkstride = 1;
+  if (r > 0) {
+    if (r <= kDecThreads) {
+      const int grp = kDecThreads / r;
+      if (tid < grp * r) { rj = tid % r; rks0 = tid / r; rkstride = grp; }
+    } else {
+      rj = tid;  // r > 128: each thread takes pairs tid, tid + 128, ... (handled in the loop)
+    }
+  }
+  // cos/sin of the per-thread key step (kstride * theta_j), exact
+  float step_c = 1.f, step_s = 0.f;
+  double inv_turns = 0.0;
+  if (rj >= 0 && r <= kDecThreads) {
+    inv_turns = rope_inv_freq_turns(rj, D, a.log2_base);
+    rope_cos_sin((double)rkstride, inv_turns, &step_c, &step_s);
+  }
+
+  // ---- chunk loader
+  auto load_chunk = [&](int chunk, int buf) {
+    const int v0 = v_lo + chunk * kCK;
+    uint16_t* kd = kbuf + buf * kCK * KST;
+    uint16_t* vd = vbuf + buf * kCK * KST;
+    for (int idx = tid; idx < kCK * PIECES; idx += kDecThreads) {
+      const int row = idx / PIECES, pc = idx % PIECES;
+      const int v = v0 + row;
+      const bool valid = v < v_hi;
+      const int pos = first + v;
+      const uint16_t* ksrc = a.k_cache;
+      const uint16_t* vsrc = a.v_cache;
+      if (valid) {
+        if (pos < len) {
+          const size_t rr = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
+          const size_t off = (((size_t)b * a.num_kv_heads + kvh) * a.capacity + rr) * D;
+          ksrc = a.k_cache + off;
+          vsrc = kv_same ? nullptr : a.v_cache + off;
+        } else {
+          const size_t off = (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
+          ksrc = a.new_k + off;
+          vsrc = kv_same ? nullptr : a.new_v + off;
+        }
+      }
+      cp_async16(kd + row * KST + pc * 8, valid ? ksrc + pc * 8 : a.k_cache, valid);
+      if (!kv_same) cp_async16(vd + row * KST + pc * 8, valid ? vsrc + pc * 8 : a.k_cache, valid);
+    }
+  };
 
   const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
-  // ---- rotated queries into shared memory
-  for (int idx = threadIdx.x; idx < G * HALF; idx += kDecThreads) {
-    const int g = idx / HALF, j = idx % HALF;
-    const int i = g / group, hh = g % group;
-    const int qpos = len + i;
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(
-        a.q + (((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh) * D);
-    float x0 = __bfloat162float(qrow[j]), x1 = __bfloat162float(qrow[j + HALF]);
-    float y0 = x0, y1 = x1;
-    if (j < a.r) {
-      float c, s;
-      rope_cos_sin((double)qpos, rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
-      y0 = x0 * c - x1 * s;
-      y1 = x0 * s + x1 * c;
-    }
-    qs[g * D + j] = y0 * scale_log2;
-    qs[g * D + j + HALF] = y1 * scale_log2;
-  }
-  __syncthreads();
+  float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) { m_run[nt][e] = -INFINITY; l_run[nt][e] = 0.f; }
+  float oacc[MTW][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < MTW; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oacc[mt][nt][e] = 0.f;
 
-  float m[kRowsPerWarp], l[kRowsPerWarp], o[kRowsPerWarp][2 * H];
-#pragma unroll
-  for (int g = 0; g < kRowsPerWarp; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 2 * H; ++e) o[g][e] = 0.f;
-  }
-  const int g0 = rg * kRowsPerWarp;
-  const int ng = warp_active ? min(kRowsPerWarp, G - g0) : 0;
+  const int nchunks = (v_hi - v_lo + kCK - 1) / kCK;
+  if (nchunks > 0) load_chunk(0, 0);
+  cp_async_commit();
 
-  // inverse frequencies (in turns) of this lane's rotated pairs
-  double inv_turns[H];
-#pragma unroll
-  for (int e = 0; e < H; ++e) inv_turns[e] = rope_inv_freq_turns(lane * H + e, D, a.log2_base);
+  for (int chunk = 0; chunk < nchunks; ++chunk) {
+    const int buf = chunk & 1;
+    if (chunk + 1 < nchunks) load_chunk(chunk + 1, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    uint16_t* kd = kbuf + buf * kCK * KST;
+    const uint16_t* vd = kv_same ? kd : vbuf + buf * kCK * KST;
+    const int v0 = v_lo + chunk * kCK;
+    const int pos0 = first + v0;
 
-  if (warp_active) {
-    for (int v = v_lo + stream_id; v < v_hi; v += streams) {
-      const int pos = first + v;
-      const uint16_t* krow;
-      const uint16_t* vrow;
-      if (pos < len) {
-        const size_t row = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
-        const size_t off = (((size_t)b * a.num_kv_heads + kvh) * a.capacity + row) * D;
-        krow = a.k_cache + off;
-        vrow = a.v_cache ? a.v_cache + off : krow;
-      } else {
-        const size_t off = (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
-        krow = a.new_k + off;
-        vrow = a.new_v ? a.new_v + off : krow;
-      }
-      float kx[2 * H], vx[2 * H];
-      if (lane < ACTIVE) {
-        const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(krow);
-        const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(vrow);
-#pragma unroll
-        for (int e = 0; e < H; ++e) {
-          kx[e] = __bfloat162float(kb[lane * H + e]);
-          kx[H + e] = __bfloat162float(kb[HALF + lane * H + e]);
-          vx[e] = __bfloat162float(vb[lane * H + e]);
-          vx[H + e] = __bfloat162float(vb[HALF + lane * H + e]);
-        }
-#pragma unroll
-        for (int e = 0; e < H; ++e) {
-          if (lane * H + e < a.r) {
-            float c, s;
-            rope_cos_sin((double)pos, inv_turns[e], &c, &s);
-            const float x0 = kx[e], x1 = kx[H + e];
-            kx[e] = x0 * c - x1 * s;
-            kx[H + e] = x0 * s + x1 * c;
+    // ---- rotated copy for scores
+    if (r > 0) {
+      if (kv_same) {
+        // non-rotated dims that share a 16-dim k-step with rotated ones are copied first
+        if (r % 16 != 0) {
+          for (int idx = tid; idx < kCK * nrk * 16; idx += kDecThreads) {
+            const int row = idx / (nrk * 16), col = idx % (nrk * 16);
+            int s = 0;
+            for (int q = 0, c = 0; q < NKS; ++q)
+              if (ks_slot[q] >= 0) { if (c == col / 16) { s = q; break; } ++c; }
+            rbuf[row * RST + col] = kd[row * KST + s * 16 + col % 16];
           }
+          __syncthreads();
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 2 * H; ++e) { kx[e] = 0.f; vx[e] = 0.f; }
       }
-#pragma unroll
-      for (int g = 0; g < kRowsPerWarp; ++g) {
-        if (g >= ng) break;
-        const int row = g0 + g;
-        const int qpos = len + row / group;
-        const float* qr = qs + (size_t)row * D;
-        float dot = 0.f;
-        if (lane < ACTIVE) {
-#pragma unroll
-          for (int e = 0; e < H; ++e) dot += qr[lane * H + e] * kx[e] + qr[HALF + lane * H + e] * kx[H + e];
+      for (int j = rj; j >= 0 && j < r; j += kDecThreads) {
+        float ac, as;
+        int ks0 = rks0, kstride = rkstride;
+        float sc = step_c, ss = step_s;
+        if (r > kDecThreads) {  // one pair per iteration over all keys
+          ks0 = 0; kstride = 1;
+          const double it = rope_inv_freq_turns(j, D, a.log2_base);
+          rope_cos_sin(1.0, it, &sc, &ss);
+          rope_cos_sin((double)pos0, it, &ac, &as);
+        } else {
+          rope_cos_sin((double)(pos0 + ks0), inv_turns, &ac, &as);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        const bool vis = pos <= qpos && (!a.is_local || pos > qpos - a.window);
-        if (!vis) continue;
-        const float mn = fmaxf(m[g], dot);
-        const float alpha = exp2f(m[g] - mn);
-        const float p = exp2f(dot - mn);
-        l[g] = l[g] * alpha + p;
-#pragma unroll
-        for (int e = 0; e < 2 * H; ++e) o[g][e] = o[g][e] * alpha + p * vx[e];
-        m[g] = mn;
+        const int sj = ks_slot[j / 16], sp = ks_slot[(j + HALF) / 16];
+        for (int u = ks0; u < kCK; u += kstride) {
+          const float x0 = bf2f(kd[u * KST + j]), x1 = bf2f(kd[u * KST + j + HALF]);
+          const uint16_t y0 = f2bf(x0 * ac - x1 * as), y1 = f2bf(x0 * as + x1 * ac);
+          if (kv_same) {
+            rbuf[u * RST + sj * 16 + (j % 16)] = y0;
+            rbuf[u * RST + sp * 16 + ((j + HALF) % 16)] = y1;
+          } else {
+            kd[u * KST + j] = y0;
+            kd[u * KST + j + HALF] = y1;
+          }
+          const float nc = ac * sc - as * ss;
+          as = ac * ss + as * sc;
+          ac = nc;
+        }
+        if (r <= kDecThreads) break;
       }
+      __syncthreads();
     }
-  }
 
-  // ---- merge the key streams of each row group in shared memory, write partials
-  const int stride = D + 2;
-  float* mine = red + (size_t)warp * kRowsPerWarp * stride;
-  for (int g = 0; g < ng; ++g) {
-    if (lane < ACTIVE) {
+    // ---- S^T = K Q^T for this warp's 16 keys
+    float sacc[NT][4];
 #pragma unroll
-      for (int e = 0; e < H; ++e) {
-        mine[g * stride + lane * H + e] = o[g][e];
-        mine[g * stride + HALF + lane * H + e] = o[g][H + e];
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+    {
+      const int krow = warp * 16 + (lane & 15);
+      const int kcol = (lane >> 4) * 8;
+#pragma unroll 4
+      for (int s = 0; s < NKS; ++s) {
+        const int slot = ks_slot[s];
+        const uint32_t aaddr = slot >= 0 ? smem_u32(rbuf + krow * RST + slot * 16 + kcol)
+                                         : smem_u32(kd + krow * KST + s * 16 + kcol);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(aaddr, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t b0, b1;
+          const int qrow = nt * 8 + (lane & 7);
+          const int qcol = s * 16 + ((lane >> 3) & 1) * 8;
+          ldsm_x2(smem_u32(qs + qrow * KST + qcol), b0, b1);
+          mma_16816(sacc[nt], a0, a1, a2, a3, b0, b1);
+        }
       }
     }
-    if (lane == 0) { mine[g * stride + D] = m[g]; mine[g * stride + D + 1] = l[g]; }
+
+    // ---- mask, chunk max per row
+    float cmax[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = nt * 8 + 2 * t + e;
+        const int qpos = len + (row < R ? row / group : 0);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int hk = 0; hk < 2; ++hk) {
+          const int key = warp * 16 + g + hk * 8;
+          const int v = v0 + key;
+          const int pos = first + v;
+          const bool vis = row < R && v < v_hi && pos <= qpos && (!a.is_local || pos > qpos - a.window);
+          float& sv = sacc[nt][hk * 2 + e];
+          sv = vis ? sv * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        cmax[nt][e] = mx;
+      }
+    }
+    if (g == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) red_max[warp * RPAD + nt * 8 + 2 * t + e] = cmax[nt][e];
+    }
+    __syncthreads();
+
+    // ---- probabilities, row sums, P to shared memory
+    float alpha[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = nt * 8 + 2 * t + e;
+        float cm = red_max[col];
+#pragma unroll
+        for (int w = 1; w < kDecWarps; ++w) cm = fmaxf(cm, red_max[w * RPAD + col]);
+        const float mn = fmaxf(m_run[nt][e], cm);
+        alpha[nt][e] = (mn == -INFINITY) ? 1.f : exp2f(m_run[nt][e] - mn);
+        const float msub = (mn == -INFINITY) ? 0.f : mn;
+        m_run[nt][e] = mn;
+        float sum = 0.f;
+#pragma unroll
+        for (int hk = 0; hk < 2; ++hk) {
+          const float p = exp2f(sacc[nt][hk * 2 + e] - msub);
+          const uint16_t pb = f2bf(p);
+          sum += bf2f(pb);
+          ps[col * PST + warp * 16 + g + hk * 8] = pb;
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 8);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+        if (g == 0) red_sum[warp * RPAD + col] = sum;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = nt * 8 + 2 * t + e;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) sum += red_sum[w * RPAD + col];
+        l_run[nt][e] = l_run[nt][e] * alpha[nt][e] + sum;
+      }
+
+    // ---- O^T += V^T P^T over this warp's head-dim slice
+    if (warp < PV_WARPS) {
+#pragma unroll
+      for (int mt = 0; mt < MTW; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          oacc[mt][nt][0] *= alpha[nt][0];
+          oacc[mt][nt][1] *= alpha[nt][1];
+          oacc[mt][nt][2] *= alpha[nt][0];
+          oacc[mt][nt][3] *= alpha[nt][1];
+        }
+#pragma unroll
+      for (int ks = 0; ks < kCK / 16; ++ks) {
+        uint32_t bfr[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int prow = nt * 8 + (lane & 7);
+          const int pcol = ks * 16 + ((lane >> 3) & 1) * 8;
+          ldsm_x2(smem_u32(ps + prow * PST + pcol), bfr[nt][0], bfr[nt][1]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MTW; ++mt) {
+          const int d0 = (warp * MTW + mt) * 16;
+          const int vrow = ks * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int vcol = d0 + ((lane >> 3) & 1) * 8;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(smem_u32(vd + vrow * KST + vcol), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(oacc[mt][nt], a0, a1, a2, a3, bfr[nt][0], bfr[nt][1]);
+        }
+      }
+    }
+    __syncthreads();  // buffers of this chunk are free for the load two chunks ahead
   }
-  __syncthreads();
+  cp_async_wait<0>();
+
+  // ---- partial O (normalised by this split's l) and log-sum-exp
   const int rows_total = a.batch * a.n_q * a.num_q_heads;
-  for (int idx = threadIdx.x; idx < G * D; idx += kDecThreads) {
-    const int row = idx / D, c = idx % D;
-    const int rgi = row / kRowsPerWarp, gi = row % kRowsPerWarp;
-    float mm = -INFINITY;
-    for (int s = 0; s < streams; ++s) {
-      const float* st = red + (size_t)(s * nrg + rgi) * kRowsPerWarp * stride + gi * stride;
-      mm = fmaxf(mm, st[D]);
-    }
-    float ll = 0.f, acc = 0.f;
-    if (mm != -INFINITY) {
-      for (int s = 0; s < streams; ++s) {
-        const float* st = red + (size_t)(s * nrg + rgi) * kRowsPerWarp * stride + gi * stride;
-        if (st[D] == -INFINITY) continue;
-        const float w = exp2f(st[D] - mm);
-        ll += w * st[D + 1];
-        acc += w * st[c];
+  if (warp < PV_WARPS) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = nt * 8 + 2 * t + e;
+        if (row >= R) continue;
+        const int i = row / group, hh = row % group;
+        const size_t orow = ((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh;
+        const float l = l_run[nt][e];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float* po = a.partial_o + ((size_t)split * rows_total + orow) * D;
+#pragma unroll
+        for (int mt = 0; mt < MTW; ++mt) {
+          const int d0 = (warp * MTW + mt) * 16;
+          po[d0 + g] = oacc[mt][nt][e] * inv;
+          po[d0 + g + 8] = oacc[mt][nt][2 + e] * inv;
+        }
+        if (warp == 0 && g == 0)
+          a.partial_lse[(size_t)split * rows_total + orow] =
+              l > 0.f ? (m_run[nt][e] + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
-    }
-    const int i = row / group, hh = row % group;
-    const size_t orow = ((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh;
-    a.partial_o[((size_t)split * rows_total + orow) * D + c] = ll > 0.f ? acc / ll : 0.f;
-    if (c == 0)
-      a.partial_lse[(size_t)split * rows_total + orow] =
-          ll > 0.f ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
   }
 }
 
-template <int D>
-static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t stream) {
-  const int group = a.num_q_heads / a.num_kv_heads;
-  const int G = group * a.n_q;
-  const size_t smem = ((size_t)G * D + (size_t)kDecWarps * kRowsPerWarp * (D + 2)) * sizeof(float);
+template <int D, int NT>
+static cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
+  const bool kv_same = a.v_cache == nullptr;
+  int nrk = 0;
+  if (kv_same)
+    for (int s = 0; s < D / 16; ++s)
+      if (s * 16 < a.r || (s * 16 < D / 2 + a.r && s * 16 + 16 > D / 2)) ++nrk;
+  const size_t smem = dec_smem_bytes<D, NT>(!kv_same, nrk);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.num_splits, a.num_kv_heads, a.batch);
-  decode_kernel<D><<<grid, kDecThreads, smem, stream>>>(a);
+  decode_tc_kernel<D, NT><<<grid, kDecThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
+// Largest supported query-row count per CTA (group * n_q) for a head dim.
+int decode_max_rows(int head_dim) { return head_dim >= 512 ? 32 : 64; }
+
+template <int D>
+static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t stream) {
+  const int R = (a.num_q_heads / a.num_kv_heads) * a.n_q;
+  if (R <= 8) return launch_decode_tc<D, 1>(a, stream);
+  if (R <= 16) return launch_decode_tc<D, 2>(a, stream);
+  if (R <= 32) return launch_decode_tc<D, 4>(a, stream);
+  if constexpr (D < 512) {
+    if (R <= 64) return launch_decode_tc<D, 8>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  const int group = a.num_q_heads / a.num_kv_heads;
-  if ((group * a.n_q + kRowsPerWarp - 1) / kRowsPerWarp > kDecWarps) return cudaErrorInvalidValue;
   switch (a.head_dim) {
     case 32: return launch_decode_d<32>(a, stream);
     case 64: return launch_decode_d<64>(a, stream);

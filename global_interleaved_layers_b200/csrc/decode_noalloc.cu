@@ -87,7 +87,9 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   if (cache_layout == GEMMA_ATTN_CACHE_CONTIGUOUS && cache_capacity < max_cache_len)
     return GEMMA_ATTN_ERR_INVALID_ARG;
   const int group = params->num_q_heads / params->num_kv_heads;
-  if ((group * n_q + 7) / 8 > 8) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  if (group * n_q > decode_max_rows(params->head_dim)) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
+    return GEMMA_ATTN_ERR_MISALIGNED;
 
   // Partials for num_splits x rows: fp32 O [splits, rows, d] then fp32 lse [splits, rows].
   const size_t rows = (size_t)batch * n_q * params->num_q_heads;

@@ -63,6 +63,7 @@ struct DecodeArgs {
   float softmax_scale;
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int decode_max_rows(int head_dim);  // largest group * n_q one decode CTA handles
 
 struct CombineArgs {
   const float* partial_o;

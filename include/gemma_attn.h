@@ -140,6 +140,8 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
  *   partial_lse [num_splits, batch * n_q * num_q_heads] float32, written (-inf for an
  *              empty split). Row index = (b * n_q + i) * num_q_heads + h.
  *   The visible keys of each sequence are cut into num_splits contiguous ranges.
+ *   Limits: (num_q_heads / num_kv_heads) * n_q <= 64 (<= 32 for head_dim 512), else
+ *   GEMMA_ATTN_ERR_UNSUPPORTED; q, new_k, new_v and the caches 16-byte aligned.
  */
 int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void* new_k,
                       const void* new_v, const void* k_cache, const void* v_cache,

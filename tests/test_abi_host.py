@@ -93,7 +93,7 @@ def test_decode_argument_errors():
     assert e.value.status == G.ERR_INVALID_ARG
     # too many query rows per KV head
     with pytest.raises(G.GemmaAttnError) as e:
-        G.gemma_attn_decode(pg, fake, fake, None, fake, None, G.CACHE_CONTIGUOUS, 64, fake, 1, 9, 10, fake, fake, 1, 0)
+        G.gemma_attn_decode(pg, fake, fake, None, fake, None, G.CACHE_CONTIGUOUS, 64, fake, 1, 5, 10, fake, fake, 1, 0)
     assert e.value.status == G.ERR_UNSUPPORTED
 
 
