@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -49,6 +50,13 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int heads, int tokens
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The two-CTA paired prefill kernel is the default; GEMMA_ATTN_NO_PAIR=1 in the
+// environment selects the single-CTA kernel (used by the tests to cover both forms).
+bool pair_kernel_enabled() {
+  const char* e = getenv("GEMMA_ATTN_NO_PAIR");
+  return !(e && e[0] == '1');
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -190,16 +198,21 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
     maps.q = maps.qs;
     maps.k = maps.ks;
     ok &= make_map(&maps.v, vpad, 64, Hkv, total_tokens, 128);
+    maps.k64 = maps.k;
+    maps.ks64 = maps.ks;
   } else {
     ok &= make_map(&maps.q, q, d, Hq, total_tokens, 128);
     ok &= make_map(&maps.k, k, d, Hkv, total_tokens, 128);
     ok &= make_map(&maps.v, global ? k : v, d, Hkv, total_tokens, 128);
+    ok &= make_map(&maps.k64, k, d, Hkv, total_tokens, 64);
     if (L.mask) {
       ok &= make_map(&maps.qs, qside, L.n_out, Hq, total_tokens, 128);
       ok &= make_map(&maps.ks, kside, L.n_out, Hkv, total_tokens, 128);
+      ok &= make_map(&maps.ks64, kside, L.n_out, Hkv, total_tokens, 64);
     } else {
       maps.qs = maps.q;
       maps.ks = maps.k;
+      maps.ks64 = maps.k64;
     }
   }
   if (!ok) return GEMMA_ATTN_ERR_LAUNCH;
@@ -210,6 +223,7 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
   a.num_q_heads = Hq; a.group = Hq / Hkv; a.head_dim = d; a.is_local = global ? 0 : 1;
   a.window = global ? 0 : params->window; a.softmax_scale = params->softmax_scale; a.rot_mask = L.mask;
   a.out_f32 = params->out_dtype == GEMMA_ATTN_OUT_F32;
+  a.pair_allowed = pair_kernel_enabled();
   cudaError_t e;
   switch (L.kd) {
     case 64: e = launch_prefill<64>(maps, a, stream); break;

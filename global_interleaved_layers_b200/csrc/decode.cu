@@ -31,14 +31,7 @@ constexpr int kDecThreads = 128;
 constexpr int kDecWarps = 4;
 constexpr int kCK = 64;  // keys per chunk
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;  // 0: zero-fill, nothing read
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+constexpr int kDecHeader = 128;  // bytes at the start of shared memory: two mbarriers, abort flag
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -84,7 +77,7 @@ struct DecSmem {
 template <int D, int NT>
 __host__ __device__ constexpr size_t dec_smem_bytes(bool separate_v, int nrk) {
   using S = DecSmem<D, NT>;
-  size_t b = 0;
+  size_t b = kDecHeader;
   b += 2ull * kCK * S::KST * 2;                        // key buffers
   if (separate_v) b += 2ull * kCK * S::KST * 2;        // value buffers
   b += (size_t)kCK * (nrk * 16 + S::kRowPad) * 2;      // rotated copy (K=V layers)
@@ -107,7 +100,6 @@ decode_tc_kernel(DecodeArgs a) {
   constexpr int MT_TOTAL = D / 16;                              // 16-dim m-tiles of O^T
   constexpr int PV_WARPS = MT_TOTAL < kDecWarps ? MT_TOTAL : kDecWarps;
   constexpr int MTW = MT_TOTAL / PV_WARPS;                      // m-tiles per PV warp
-  constexpr int PIECES = D / 8;                                 // 16-byte pieces per row
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -128,9 +120,15 @@ decode_tc_kernel(DecodeArgs a) {
     for (int s = 0; s < NKS; ++s)
       if (s * 16 < r || (s * 16 < HALF + r && s * 16 + 16 > HALF)) ++nrk;
   const int RST = nrk * 16 + S::kRowPad;
+  uint32_t rot_bits = 0;  // bit s: k-step s of the scores reads the rotated copy
+  if (kv_same)
+    for (int s = 0; s < NKS; ++s)
+      if (s * 16 < r || (s * 16 < HALF + r && s * 16 + 16 > HALF)) rot_bits |= 1u << s;
 
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint16_t* kbuf = reinterpret_cast<uint16_t*>(dsm);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(dsm);          // [2], one per chunk buffer
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + 16);
+  uint16_t* kbuf = reinterpret_cast<uint16_t*>(dsm + kDecHeader);
   uint16_t* vbuf = kbuf + 2 * kCK * KST;
   uint16_t* rbuf = kv_same ? vbuf : vbuf + 2 * kCK * KST;
   uint16_t* qs = rbuf + kCK * RST;
@@ -139,6 +137,12 @@ decode_tc_kernel(DecodeArgs a) {
   float* red_sum = red_max + kDecWarps * RPAD;
   int* ks_slot = reinterpret_cast<int*>(red_sum + kDecWarps * RPAD);
 
+  if (tid == 0) {
+    mbar_init(&full_bar[0], 1);
+    mbar_init(&full_bar[1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
   if (tid < NKS) {
     int slot = -1;
     if (kv_same) {
@@ -190,32 +194,32 @@ decode_tc_kernel(DecodeArgs a) {
     rope_cos_sin((double)rkstride, inv_turns, &step_c, &step_s);
   }
 
-  // ---- chunk loader
-  auto load_chunk = [&](int chunk, int buf) {
+  // ---- chunk loader: warp 0 issues one bulk copy per key (and value) row of the chunk
+  // into the padded buffer rows; the copies complete on the buffer's mbarrier.
+  auto issue_chunk = [&](int chunk, int buf) {
     const int v0 = v_lo + chunk * kCK;
+    const int nvalid = min(kCK, v_hi - v0);
     uint16_t* kd = kbuf + buf * kCK * KST;
     uint16_t* vd = vbuf + buf * kCK * KST;
-    for (int idx = tid; idx < kCK * PIECES; idx += kDecThreads) {
-      const int row = idx / PIECES, pc = idx % PIECES;
-      const int v = v0 + row;
-      const bool valid = v < v_hi;
-      const int pos = first + v;
-      const uint16_t* ksrc = a.k_cache;
-      const uint16_t* vsrc = a.v_cache;
-      if (valid) {
-        if (pos < len) {
-          const size_t rr = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
-          const size_t off = (((size_t)b * a.num_kv_heads + kvh) * a.capacity + rr) * D;
-          ksrc = a.k_cache + off;
-          vsrc = kv_same ? nullptr : a.v_cache + off;
-        } else {
-          const size_t off = (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
-          ksrc = a.new_k + off;
-          vsrc = kv_same ? nullptr : a.new_v + off;
-        }
+    fence_proxy_async_smem();  // earlier generic accesses to this buffer come first
+    if (lane == 0) mbar_arrive_expect_tx(&full_bar[buf], (uint32_t)(nvalid * D * 2 * (kv_same ? 1 : 2)));
+    __syncwarp();
+    for (int row = lane; row < nvalid; row += 32) {
+      const int pos = first + v0 + row;
+      const uint16_t* ksrc;
+      const uint16_t* vsrc;
+      if (pos < len) {
+        const size_t rr = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
+        const size_t off = (((size_t)b * a.num_kv_heads + kvh) * a.capacity + rr) * D;
+        ksrc = a.k_cache + off;
+        vsrc = kv_same ? nullptr : a.v_cache + off;
+      } else {
+        const size_t off = (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
+        ksrc = a.new_k + off;
+        vsrc = kv_same ? nullptr : a.new_v + off;
       }
-      cp_async16(kd + row * KST + pc * 8, valid ? ksrc + pc * 8 : a.k_cache, valid);
-      if (!kv_same) cp_async16(vd + row * KST + pc * 8, valid ? vsrc + pc * 8 : a.k_cache, valid);
+      bulk_load(kd + row * KST, ksrc, D * 2, &full_bar[buf]);
+      if (!kv_same) bulk_load(vd + row * KST, vsrc, D * 2, &full_bar[buf]);
     }
   };
 
@@ -234,19 +238,30 @@ decode_tc_kernel(DecodeArgs a) {
       for (int e = 0; e < 4; ++e) oacc[mt][nt][e] = 0.f;
 
   const int nchunks = (v_hi - v_lo + kCK - 1) / kCK;
-  if (nchunks > 0) load_chunk(0, 0);
-  cp_async_commit();
+  __syncthreads();  // barrier init and the rotated queries are visible to every thread
+  if (warp == 0 && nchunks > 0) issue_chunk(0, 0);
+  int in_flight = nchunks > 0 ? 0 : -1;  // chunk whose copies are issued but not yet waited on
 
   for (int chunk = 0; chunk < nchunks; ++chunk) {
     const int buf = chunk & 1;
-    if (chunk + 1 < nchunks) load_chunk(chunk + 1, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
+    if (warp == 0 && chunk + 1 < nchunks) issue_chunk(chunk + 1, buf ^ 1);
+    const bool ok = mbar_wait(&full_bar[buf], (uint32_t)(chunk >> 1) & 1u, abort_flag);
+    in_flight = chunk + 1 < nchunks ? chunk + 1 : -1;
+    if (__syncthreads_or(!ok)) break;
     uint16_t* kd = kbuf + buf * kCK * KST;
-    const uint16_t* vd = kv_same ? kd : vbuf + buf * kCK * KST;
+    uint16_t* vdw = kv_same ? kd : vbuf + buf * kCK * KST;
+    const uint16_t* vd = vdw;
     const int v0 = v_lo + chunk * kCK;
     const int pos0 = first + v0;
+    const int nvalid = min(kCK, v_hi - v0);
+    if (nvalid < kCK) {  // rows past the split end: zero, so that P = 0 meets finite values
+      for (int idx = tid; idx < (kCK - nvalid) * (D / 8); idx += kDecThreads) {
+        const int row = nvalid + idx / (D / 8), c8 = idx % (D / 8);
+        *reinterpret_cast<uint4*>(kd + row * KST + c8 * 8) = make_uint4(0, 0, 0, 0);
+        if (!kv_same) *reinterpret_cast<uint4*>(vdw + row * KST + c8 * 8) = make_uint4(0, 0, 0, 0);
+      }
+      __syncthreads();
+    }
 
     // ---- rotated copy for scores
     if (r > 0) {
@@ -276,6 +291,7 @@ decode_tc_kernel(DecodeArgs a) {
           rope_cos_sin((double)(pos0 + ks0), inv_turns, &ac, &as);
         }
         const int sj = ks_slot[j / 16], sp = ks_slot[(j + HALF) / 16];
+#pragma unroll 4
         for (int u = ks0; u < kCK; u += kstride) {
           const float x0 = bf2f(kd[u * KST + j]), x1 = bf2f(kd[u * KST + j + HALF]);
           const uint16_t y0 = f2bf(x0 * ac - x1 * as), y1 = f2bf(x0 * as + x1 * ac);
@@ -295,31 +311,39 @@ decode_tc_kernel(DecodeArgs a) {
       __syncthreads();
     }
 
-    // ---- S^T = K Q^T for this warp's 16 keys
+    // ---- S^T = K Q^T for this warp's 16 keys. Two accumulator sets (even / odd
+    // k-steps) halve the dependent mma chain; the rotated-slot lookup uses a register
+    // bitmask so no shared-memory load sits on the address path.
     float sacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
     {
+      float sacc2[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { sacc[nt][e] = 0.f; sacc2[nt][e] = 0.f; }
       const int krow = warp * 16 + (lane & 15);
       const int kcol = (lane >> 4) * 8;
-#pragma unroll 4
+      const uint32_t kbase = smem_u32(kd + krow * KST + kcol);
+      const uint32_t rbase = smem_u32(rbuf + krow * RST + kcol);
+      const uint32_t qbase = smem_u32(qs + (lane & 7) * KST + ((lane >> 3) & 1) * 8);
+#pragma unroll
       for (int s = 0; s < NKS; ++s) {
-        const int slot = ks_slot[s];
-        const uint32_t aaddr = slot >= 0 ? smem_u32(rbuf + krow * RST + slot * 16 + kcol)
-                                         : smem_u32(kd + krow * KST + s * 16 + kcol);
+        const bool rot = (rot_bits >> s) & 1u;
+        const int slot = __popc(rot_bits & ((1u << s) - 1u));
+        const uint32_t aaddr = rot ? rbase + slot * 32 : kbase + s * 32;
         uint32_t a0, a1, a2, a3;
         ldsm_x4(aaddr, a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           uint32_t b0, b1;
-          const int qrow = nt * 8 + (lane & 7);
-          const int qcol = s * 16 + ((lane >> 3) & 1) * 8;
-          ldsm_x2(smem_u32(qs + qrow * KST + qcol), b0, b1);
-          mma_16816(sacc[nt], a0, a1, a2, a3, b0, b1);
+          ldsm_x2(qbase + (nt * 8 * KST + s * 16) * 2, b0, b1);
+          mma_16816((s & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, b0, b1);
         }
       }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
     }
 
     // ---- mask, chunk max per row
@@ -429,7 +453,12 @@ decode_tc_kernel(DecodeArgs a) {
     }
     __syncthreads();  // buffers of this chunk are free for the load two chunks ahead
   }
-  cp_async_wait<0>();
+  // Copies still in flight after an early exit land before the CTA leaves.
+  if (in_flight >= 0 && tid == 0) {
+    const uint32_t par = (uint32_t)(in_flight >> 1) & 1u;
+    unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(&full_bar[in_flight & 1], par) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+  }
 
   // ---- partial O (normalised by this split's l) and log-sum-exp
   const int rows_total = a.batch * a.n_q * a.num_q_heads;

@@ -22,11 +22,13 @@ struct PrefillArgs {
   int window;
   float softmax_scale;
   int out_f32;        // 1: write fp32 output, 0: bf16
+  int pair_allowed;   // 1: use the two-CTA paired kernel where the shape permits
   uint32_t rot_mask;  // bit c set: key/query chunk c (64 dims) is read from the rotated side copy
 };
 
 struct PrefillMaps {
-  CUtensorMap q, qs, k, ks, v;
+  CUtensorMap q, qs, k, ks, v;   // 128-row boxes
+  CUtensorMap k64, ks64;         // 64-row boxes: one CTA's half of a key tile (paired form)
 };
 
 template <int D>

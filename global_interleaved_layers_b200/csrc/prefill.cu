@@ -1,29 +1,36 @@
 // prefill.cu -- flash-style causal attention for Gemma-4-style local (sliding
 // window) and global (K=V, p-RoPE) layers on sm_100a.
 //
-// One CTA computes a 128-row query tile of one query head against the key tiles
-// its rows can see (global: all earlier keys; local: the last W keys; "Visual
-// guide to Gemma 4", section "Interleaving Layers"). Fully masked key tiles are
-// never loaded; only tiles that straddle the diagonal or the window edge are masked.
+// A work unit is a 128-row query tile of one query head against the key tiles its
+// rows can see (global: all earlier keys; local: the last W keys; "Visual guide to
+// Gemma 4", section "Interleaving Layers"). Fully masked key tiles are never loaded;
+// only tiles that straddle the diagonal, the window edge or a sequence end are masked.
 //
-// Roles (192 threads):
-//   warp 0     TMA producer: the Q tile once, then 16 KB chunks (128 keys x 64
-//              dims, 128-byte swizzle) of K and V through a ring of stages.
-//   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score
-//              buffers (tcgen05.mma, both operands in shared memory), then
-//              O += P V with P read from TMEM and V from the ring.
-//   warps 2-5  softmax: one query row per thread; online softmax in fp32 with
-//              the running max only raised when it grows by more than 2^8, P written
-//              back to TMEM as bf16 over the scores, epilogue O / l -> bf16.
+// Roles (192 threads per CTA):
+//   warp 0     TMA producer: the Q tile once, then 16 KB stages of K and V through a
+//              ring (128-byte swizzle).
+//   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score buffers
+//              (tcgen05.mma, both operands in shared memory), then O += P V with P read
+//              from TMEM and V from the ring.
+//   warps 2-5  softmax: one query row per thread; online softmax in fp32 with the
+//              running max only raised when it grows by more than 2^8, P written back to
+//              TMEM as bf16 over the scores, epilogue O / l.
 // The MMA order is S(j), PV(j-1), S(j+1), PV(j), ... so the tensor core works on
 // S(j+1) while the softmax warps turn S(j) into P(j).
 //
-// Global layers: the single K=V tensor feeds both operands. Key chunks that hold
-// rotated dimensions come from a rotated side copy (workspace); every other key
-// chunk and every value chunk are read from the un-rotated tensor ("Visual guide
-// to Gemma 4", sections "K=V technique" and "p-RoPE"). With head_dim 512 the
-// 128 x 512 fp32 output tile would fill all of TMEM, so two CTAs each own one
-// 256-column half of the output and both compute the full score tile.
+// Paired form (PAIR): the two query heads of a GQA pair share every K and V tile. Two
+// CTAs on two SMs form a cluster; the even CTA issues 256-row MMAs (tcgen05 cta_group::2)
+// whose rows 0-127 are its head and rows 128-255 the odd CTA's head. Each CTA loads only
+// half of every K tile (64 of the 128 keys) and half of every V stage's columns, so the
+// bytes each SM pulls from L2 per FLOP are halved; the loads of both CTAs complete on the
+// even CTA's barriers, and the paired MMA commits signal both CTAs.
+//
+// Global layers: the single K=V tensor feeds both operands. Key chunks that hold rotated
+// dimensions come from a rotated side copy (workspace); every other key chunk and every
+// value chunk are read from the un-rotated tensor ("Visual guide to Gemma 4", sections
+// "K=V technique" and "p-RoPE"). With head_dim 512 the 128 x 512 fp32 output tile would
+// fill all of TMEM, so two work units each own one 256-column half of the output and both
+// compute the full score tile.
 #include "common.cuh"
 #include "kernels.h"
 #include "tile_plan.h"
@@ -35,23 +42,29 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kChunk = 64;                   // dims per TMA box / swizzle row
-constexpr int kStageBytes = kBN * 128;       // 128 rows x 128 bytes
+constexpr int kStageBytes = 16384;           // one ring stage
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
-template <int D>
+template <int D, bool PAIR>
 struct PrefillCfg {
-  static constexpr int kDv = D > 256 ? 256 : D;             // output columns per CTA
-  static constexpr int kSplit = D / kDv;                      // CTAs per (tile, head)
+  static constexpr int kDv = D > 256 ? 256 : D;             // output columns per work unit
+  static constexpr int kSplit = D / kDv;                      // work units per (tile, head)
   static constexpr int kQChunks = D / kChunk;
   static constexpr int kVChunks = kDv / kChunk;
   static constexpr int kQBytes = kQChunks * kStageBytes;
   static constexpr int kStages = D >= 512 ? 6 : 8;
+  // Single CTA: a K stage is one 64-dim chunk of 128 keys; a V stage one 64-dim chunk.
+  // Pair: a K stage is two 64-dim chunks of this CTA's 64 keys; a V stage one 64-dim
+  // chunk of 128 keys (the pair's two CTAs hold adjacent chunks).
+  static constexpr int kKStages = PAIR ? kQChunks / 2 : kQChunks;
+  static constexpr int kVStages = PAIR ? kVChunks / 2 : kVChunks;
   static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
   static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(!PAIR || D >= 128, "paired form needs at least two 64-dim chunks");
 };
 
 struct __align__(8) Barriers {
@@ -68,14 +81,22 @@ struct __align__(8) Barriers {
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
+// Waits that may be satisfied by the other CTA of a pair use cluster-scope acquire.
+template <bool PAIR>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if constexpr (PAIR) return mbar_wait_cluster(bar, parity, abort);
+  else return mbar_wait(bar, parity, abort);
+}
+
 }  // namespace
 
-template <int D>
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap qs_map,
                const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap ks_map,
-               const __grid_constant__ CUtensorMap v_map, PrefillArgs args) {
-  using Cfg = PrefillCfg<D>;
+               const __grid_constant__ CUtensorMap v_map, const __grid_constant__ CUtensorMap k64_map,
+               const __grid_constant__ CUtensorMap ks64_map, PrefillArgs args) {
+  using Cfg = PrefillCfg<D, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_smem = smem;
@@ -86,8 +107,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
   const int lane = threadIdx.x & 31;
 
   // ---- which work unit ----
-  const int head = blockIdx.x / Cfg::kSplit;
-  const int vpart = blockIdx.x % Cfg::kSplit;
+  // blockIdx.x = (head_unit * kSplit + vpart) [* 2 + rank in the pair]
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit_x = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int vpart = unit_x % Cfg::kSplit;
+  const int head = PAIR ? (unit_x / Cfg::kSplit) * 2 + (int)rank : unit_x / Cfg::kSplit;
   const int slot = blockIdx.y;
   const int seq = slot % args.num_seqs;
   const int qt = args.max_qtiles - 1 - slot / args.num_seqs;  // heaviest tiles first
@@ -95,6 +120,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
   const int len = args.cu_seqlens[seq + 1] - tok0;
   if (qt == 0 && vpart == 0 && head == 0 && threadIdx.x == 0 && (len > args.max_seqlen || len < 1))
     atomicOr(&g_status, kStatusSeqlen);
+  // Both CTAs of a pair share (seq, qt), so they leave here together, before any
+  // cluster-wide synchronisation.
   if (qt * kBM >= len) return;
   const int row0 = qt * kBM;
   const int kvh = head / args.group;
@@ -104,20 +131,36 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
   const int ntiles = kt_hi - kt_lo;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->s_full[b], 1); mbar_init(&bars->p_full[b], 128); }
+    const uint32_t load_arrivals = PAIR ? 2u : 1u;  // pair: both producers register their bytes
+    mbar_init(&bars->q_full, load_arrivals);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], PAIR ? 256 : 128);
+    }
     mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->mma_done, 1);
-    for (int s = 0; s < Cfg::kStages; ++s) { mbar_init(&bars->ring_full[s], 1); mbar_init(&bars->ring_empty[s], 1); }
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&bars->ring_full[s], load_arrivals);
+      mbar_init(&bars->ring_empty[s], 1);
+    }
     bars->abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&bars->tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&bars->tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {  // the peer's barriers are initialised before any remote arrival
+    __syncwarp();
+    cluster_sync_all();
+  }
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
@@ -125,118 +168,158 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tensormap(&q_map); prefetch_tensormap(&k_map); prefetch_tensormap(&v_map);
-      if (args.rot_mask) { prefetch_tensormap(&qs_map); prefetch_tensormap(&ks_map); }
-      mbar_arrive_expect_tx(&bars->q_full, Cfg::kQBytes);
+      prefetch_tensormap(&q_map); prefetch_tensormap(&v_map);
+      if (PAIR) prefetch_tensormap(&k64_map); else prefetch_tensormap(&k_map);
+      if (args.rot_mask) { prefetch_tensormap(&qs_map); prefetch_tensormap(PAIR ? &ks64_map : &ks_map); }
+      // Register `bytes` on the load barrier that counts them: this CTA's own barrier, or
+      // in the paired form the even CTA's (the odd CTA arrives remotely).
+      auto expect = [&](uint64_t* bar, uint32_t bytes) {
+        if (!PAIR || leader) mbar_arrive_expect_tx(bar, bytes);
+        else mbar_arrive_expect_tx_cluster(smem_u32(bar) & kPeerBitMask, bytes);
+      };
+      auto load = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
+        if constexpr (PAIR) tma_load_3d_pair(dst, map, bar, c0, c1, c2);
+        else tma_load_3d(dst, map, bar, c0, c1, c2);
+      };
+      auto rot_idx = [&](int c) { return __popc(args.rot_mask & ((1u << c) - 1)); };
+
+      expect(&bars->q_full, Cfg::kQBytes);
       for (int c = 0; c < Cfg::kQChunks; ++c) {
-        if ((args.rot_mask >> c) & 1) {
-          int ridx = __popc(args.rot_mask & ((1u << c) - 1));
-          tma_load_3d(q_smem + c * kStageBytes, &qs_map, &bars->q_full, ridx * kChunk, head, tok0 + row0);
-        } else {
-          tma_load_3d(q_smem + c * kStageBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
-        }
+        if ((args.rot_mask >> c) & 1) load(q_smem + c * kStageBytes, &qs_map, &bars->q_full, rot_idx(c) * kChunk, head, tok0 + row0);
+        else load(q_smem + c * kStageBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
       }
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
       bool ok = true;
       for (int jj = 0; jj <= ntiles && ok; ++jj) {
-        if (jj < ntiles) {  // K chunks of tile jj
+        if (jj < ntiles) {  // K stages of tile jj
           const int key0 = tok0 + (kt_lo + jj) * kBN;
-          for (int c = 0; c < Cfg::kQChunks && ok; ++c) {
+          for (int s = 0; s < Cfg::kKStages && ok; ++s) {
             ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
             if (!ok) break;
-            mbar_arrive_expect_tx(&bars->ring_full[st], kStageBytes);
-            if ((args.rot_mask >> c) & 1) {
-              int ridx = __popc(args.rot_mask & ((1u << c) - 1));
-              tma_load_3d(ring + st * kStageBytes, &ks_map, &bars->ring_full[st], ridx * kChunk, kvh, key0);
+            expect(&bars->ring_full[st], kStageBytes);
+            uint8_t* dst = ring + st * kStageBytes;
+            if constexpr (PAIR) {
+              // chunks 2s and 2s+1 of this CTA's 64 keys
+              for (int sub = 0; sub < 2; ++sub) {
+                const int c = 2 * s + sub;
+                if ((args.rot_mask >> c) & 1)
+                  load(dst + sub * 8192, &ks64_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh, key0 + 64 * (int)rank);
+                else
+                  load(dst + sub * 8192, &k64_map, &bars->ring_full[st], c * kChunk, kvh, key0 + 64 * (int)rank);
+              }
             } else {
-              tma_load_3d(ring + st * kStageBytes, &k_map, &bars->ring_full[st], c * kChunk, kvh, key0);
+              const int c = s;
+              if ((args.rot_mask >> c) & 1) load(dst, &ks_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh, key0);
+              else load(dst, &k_map, &bars->ring_full[st], c * kChunk, kvh, key0);
             }
             next();
           }
         }
-        if (jj >= 1) {  // V chunks of tile jj-1 (this CTA's output columns)
+        if (jj >= 1) {  // V stages of tile jj-1 (this unit's output columns)
           const int key0 = tok0 + (kt_lo + jj - 1) * kBN;
-          for (int c = 0; c < Cfg::kVChunks && ok; ++c) {
+          for (int s = 0; s < Cfg::kVStages && ok; ++s) {
             ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
             if (!ok) break;
-            mbar_arrive_expect_tx(&bars->ring_full[st], kStageBytes);
-            tma_load_3d(ring + st * kStageBytes, &v_map, &bars->ring_full[st],
-                        vpart * Cfg::kDv + c * kChunk, kvh, key0);
+            expect(&bars->ring_full[st], kStageBytes);
+            const int c = PAIR ? 2 * s + (int)rank : s;
+            load(ring + st * kStageBytes, &v_map, &bars->ring_full[st], vpart * Cfg::kDv + c * kChunk, kvh, key0);
             next();
           }
         }
       }
-      // Let every copy this thread issued land before the CTA can exit: the last
-      // kStages loads are the only ones that may still be in flight. (st, ph) is the
+      // Let the copies counted on this CTA's barriers land before the CTA can exit: the
+      // last kStages loads are the only ones that may still be in flight. (st, ph) is the
       // next slot to fill; each slot's most recent fill completed the phase of parity
-      // ph ^ 1 (the wrap inside next() flips ph for the slots filled this round).
-      for (int s = 0; s < Cfg::kStages; ++s) {
-        if (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u)) {
-          unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+      // ph ^ 1 (the wrap inside next() flips ph for the slots filled this round). In the
+      // paired form the odd CTA's copies complete on the even CTA's barriers, whose MMA
+      // consumes every one of them before the final cluster barrier.
+      if (!PAIR || leader) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
+          if (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u)) {
+            unsigned long long t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+          }
+          next();
+          (void)s;
         }
-        next();
-        (void)s;
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = umma_idesc_bf16(kBM, kBN, 0, 0);
-      const uint32_t idesc_pv = umma_idesc_bf16(kBM, kChunk, 0, 1);
-      const uint32_t q_base = smem_u32(q_smem);
-      const uint32_t r_base = smem_u32(ring);
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      constexpr int M = PAIR ? 2 * kBM : kBM;
+      constexpr int PV_N = PAIR ? 2 * kChunk : kChunk;
+      const uint32_t idesc_qk = umma_idesc_bf16(M, kBN, 0, 0);
+      const uint32_t idesc_pv = umma_idesc_bf16(M, PV_N, 0, 1);
+      // descriptors of stage 0 / Q chunk 0; other stages and k-steps are offsets of
+      // (bytes >> 4) in the low start-address field
+      const uint64_t q_desc0 = sdesc_sw128(smem_u32(q_smem), 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(smem_u32(ring), 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(ring), kStageBytes, 1024);
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
+      bool ok = wait_bar<PAIR>(&bars->q_full, 0, abort_flag);
       for (int jj = 0; jj <= ntiles && ok; ++jj) {
         if (jj < ntiles) {
           const int b = jj & 1;
           const uint32_t s_col = b ? kColS1 : kColS0;
-          if (jj >= 2) ok = mbar_wait(&bars->pv_done, (uint32_t)(jj - 2) & 1u, abort_flag);
+          if (jj >= 2) ok = wait_bar<PAIR>(&bars->pv_done, (uint32_t)(jj - 2) & 1u, abort_flag);
           tc_fence_after();
-          for (int c = 0; c < Cfg::kQChunks && ok; ++c) {
-            ok = mbar_wait(&bars->ring_full[st], ph, abort_flag);
+          for (int s = 0; s < Cfg::kKStages && ok; ++s) {
+            ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
             if (!ok) break;
             tc_fence_after();
+            const uint64_t kd = k_desc0 + (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk) {
-              uint64_t a = sdesc_sw128(q_base + c * kStageBytes + kk * 32, 16, 1024);
-              uint64_t bdesc = sdesc_sw128(r_base + st * kStageBytes + kk * 32, 16, 1024);
-              umma_ss(tmem + s_col, a, bdesc, idesc_qk, (c | kk) != 0);
+            for (int sub = 0; sub < (PAIR ? 2 : 1); ++sub) {
+              const int c = PAIR ? 2 * s + sub : s;
+              const uint64_t qd = q_desc0 + (uint64_t)((c * kStageBytes) >> 4);
+              const uint64_t kds = kd + (uint64_t)((sub * 8192) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kChunk / 16; ++kk) {
+                if constexpr (PAIR) umma_ss_pair(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
+                else umma_ss(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
+              }
             }
-            umma_commit(&bars->ring_empty[st]);
+            if constexpr (PAIR) umma_commit_pair_both(&bars->ring_empty[st]);
+            else umma_commit(&bars->ring_empty[st]);
             next();
           }
           if (!ok) break;
-          umma_commit(&bars->s_full[b]);
+          if constexpr (PAIR) umma_commit_pair_both(&bars->s_full[b]);
+          else umma_commit(&bars->s_full[b]);
         }
         if (jj >= 1) {
           const int pj = jj - 1;
           const int pb = pj & 1;
           const uint32_t p_col = pb ? kColS1 : kColS0;
-          ok = mbar_wait(&bars->p_full[pb], (uint32_t)(pj >> 1) & 1u, abort_flag);
+          ok = wait_bar<PAIR>(&bars->p_full[pb], (uint32_t)(pj >> 1) & 1u, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          for (int c = 0; c < Cfg::kVChunks && ok; ++c) {
-            ok = mbar_wait(&bars->ring_full[st], ph, abort_flag);
+          for (int s = 0; s < Cfg::kVStages && ok; ++s) {
+            ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
             if (!ok) break;
             tc_fence_after();
+            const uint64_t vd = v_desc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint32_t o_col = kColO + s * PV_N;
 #pragma unroll
             for (int kk = 0; kk < kBN / 16; ++kk) {
-              uint64_t bdesc = sdesc_sw128(r_base + st * kStageBytes + kk * 2048, kStageBytes, 1024);
-              umma_ts(tmem + kColO + c * kChunk, tmem + p_col + kk * 8, bdesc, idesc_pv, (pj | kk) != 0);
+              if constexpr (PAIR) umma_ts_pair(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, (pj | kk) != 0);
+              else umma_ts(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, (pj | kk) != 0);
             }
-            umma_commit(&bars->ring_empty[st]);
+            if constexpr (PAIR) umma_commit_pair_both(&bars->ring_empty[st]);
+            else umma_commit(&bars->ring_empty[st]);
             next();
           }
           if (!ok) break;
-          umma_commit(&bars->pv_done);
+          if constexpr (PAIR) umma_commit_pair_both(&bars->pv_done);
+          else umma_commit(&bars->pv_done);
         }
       }
       // All MMAs issued by this thread are complete once mma_done fires.
-      umma_commit(&bars->mma_done);
+      if constexpr (PAIR) umma_commit_pair_local(&bars->mma_done);
+      else umma_commit(&bars->mma_done);
       unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(&bars->mma_done, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
     }
@@ -253,7 +336,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     for (int jj = 0; jj < ntiles && ok; ++jj) {
       const int b = jj & 1;
       const uint32_t s_col = b ? kColS1 : kColS0;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float t[kBN];
@@ -283,12 +366,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           m_tile = fmaxf(m_tile, t[c]);
         }
       }
-      // O may only be touched once PV(jj-1) has finished.
-      if (jj >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-      }
       // Raise the running max only when it grows by more than 2^8 (or was empty); P
       // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
       float alpha = 1.f;
@@ -300,6 +377,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           rescale_o = true;
         }
         m_used = m_tile;
+      }
+      // P(jj) goes over S(jj) right away: that buffer's previous P (tile jj-2) was consumed
+      // by PV(jj-2), which finished before S(jj) was computed. Only the O rescale has to
+      // wait for PV(jj-1), so the exponentials stay off the PV -> softmax -> PV chain.
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+      uint32_t p[kBN / 2];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN / 2; ++c) {
+        float p0 = fast_exp2(t[2 * c] - m_sub);
+        float p1 = fast_exp2(t[2 * c + 1] - m_sub);
+        rs += p0 + p1;
+        p[c] = pack_bf16x2(p0, p1);
+      }
+      l_sum += rs;
+      tmem_st_x32(tmem + lane_off + s_col, p);
+      tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
+      // O may only be touched once PV(jj-1) has finished.
+      if (jj >= 1) {
+        ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag));
+        if (!ok) {
+          tmem_st_wait();  // the P stores land before the teardown frees TMEM
+          break;
+        }
+        tc_fence_after();
       }
       // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
       // lane needs it, each lane with its own factor (1 for lanes that do not).
@@ -314,25 +416,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
         }
       }
-      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t p[kBN / 2];
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < kBN / 2; ++c) {
-        float p0 = fast_exp2(t[2 * c] - m_sub);
-        float p1 = fast_exp2(t[2 * c + 1] - m_sub);
-        rs += p0 + p1;
-        p[c] = pack_bf16x2(p0, p1);
-      }
-      l_sum += rs;
-      tmem_st_x32(tmem + lane_off + s_col, p);
-      tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[b]);
+      if (!PAIR || leader) mbar_arrive(&bars->p_full[b]);
+      else mbar_arrive_cluster(smem_u32(&bars->p_full[b]) & kPeerBitMask);
     }
     if (ok && ntiles > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag));
     if (ok) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -369,34 +459,58 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
+  // A pair leaves together: no remote arrival or copy may target a CTA that has exited.
+  if constexpr (PAIR) {
+    __syncwarp();
+    cluster_sync_all();
+  }
   if (warp == 1) {
     // tcgen05.dealloc is warp-collective: lane 0 ran the MMA loop alone, so the warp
     // reconverges explicitly before the whole warp frees the columns.
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-template <int D>
-int prefill_smem_bytes() { return PrefillCfg<D>::kSmemBytes; }
-
-template <int D>
-cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
-  using Cfg = PrefillCfg<D>;
+template <int D, bool PAIR>
+cudaError_t launch_prefill_t(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
+  using Cfg = PrefillCfg<D, PAIR>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(args.num_q_heads * Cfg::kSplit, args.num_seqs * args.max_qtiles);
-  prefill_kernel<D><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(maps.q, maps.qs, maps.k, maps.ks, maps.v, args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(args.num_q_heads * Cfg::kSplit, args.num_seqs * args.max_qtiles);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, PAIR>, maps.q, maps.qs, maps.k, maps.ks, maps.v, maps.k64,
+                            maps.ks64, args);
 }
 
-int prefill_out_split(int D) { return D > 256 ? D / 256 : 1; }
+// The paired form runs when a pair of query heads shares a KV head (even GQA group)
+// and the head dim has at least two 64-dim chunks.
+template <int D>
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
+  if constexpr (D >= 128) {
+    if (args.group % 2 == 0 && args.pair_allowed) return launch_prefill_t<D, true>(maps, args, stream);
+  }
+  return launch_prefill_t<D, false>(maps, args, stream);
+}
 
 template cudaError_t launch_prefill<64>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);
 template cudaError_t launch_prefill<128>(const PrefillMaps&, const PrefillArgs&, cudaStream_t);

@@ -10,51 +10,76 @@
 
 namespace gattn {
 
-// One thread per (token, output column); the angle is computed once and applied to
-// every head of that token.
+namespace {
+
+// Column of the side copy that holds head dimension `dim`, or -1 when dim's 64-dim chunk
+// is not copied.
+__device__ __forceinline__ int side_col(uint32_t chunk_mask, int dim) {
+  const int c = dim >> 6;
+  if (!((chunk_mask >> c) & 1u)) return -1;
+  return __popc(chunk_mask & ((1u << c) - 1u)) * 64 + (dim & 63);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+}  // namespace
+
+// One thread per (token, group of 8 consecutive pairs j0..j0+7): it computes the 8
+// angles once and rotates those pairs in every head of the token with 16-byte loads
+// and stores of both halves (dims j0.. and j0 + d/2 ..).
 __global__ void rope_side_kernel(RopeArgs a) {
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long total = (long long)a.tokens * a.n_out;
-  if (idx >= total) return;
-  const int tok = (int)(idx / a.n_out);
-  const int o = (int)(idx % a.n_out);
-  // o-th copied column -> dimension of the (padded) head
-  int want = o / 64, chunk = 0;
-  for (int c = 0; c < 32; ++c) {
-    if ((a.chunk_mask >> c) & 1u) {
-      if (want == 0) { chunk = c; break; }
-      --want;
-    }
-  }
-  const int dim = chunk * 64 + (o % 64);
   const int half = a.d / 2;
-  uint16_t* dst = a.dst + (size_t)tok * a.heads * a.n_out + o;
-  const uint16_t* src = a.src + (size_t)tok * a.heads * a.d;
-  if (dim >= a.d) {
-    for (int h = 0; h < a.heads; ++h) dst[(size_t)h * a.n_out] = 0;
-    return;
+  const int groups = half / 8;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.tokens * groups) return;
+  const int tok = (int)(idx / groups);
+  const int j0 = (int)(idx % groups) * 8;
+  const int col0 = side_col(a.chunk_mask, j0);
+  const int col1 = side_col(a.chunk_mask, j0 + half);
+  float c[8], s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    c[e] = 1.f;
+    s[e] = 0.f;
+    if (j0 + e < a.r) rope_cos_sin((double)a.positions[tok], rope_inv_freq_turns(j0 + e, a.d, a.log2_base), &c[e], &s[e]);
   }
-  const int j = dim < half ? dim : dim - half;
-  if (j >= a.r) {
-    for (int h = 0; h < a.heads; ++h) dst[(size_t)h * a.n_out] = src[(size_t)h * a.d + dim];
-    return;
-  }
-  float c, s;
-  rope_cos_sin((double)a.positions[tok], rope_inv_freq_turns(j, a.d, a.log2_base), &c, &s);
+  const bool pad = a.d < 64 && j0 == 0;  // this thread also zeroes the padding columns d .. 63
   for (int h = 0; h < a.heads; ++h) {
-    const __nv_bfloat16* row = reinterpret_cast<const __nv_bfloat16*>(src + (size_t)h * a.d);
-    const float x0 = __bfloat162float(row[j]);
-    const float x1 = __bfloat162float(row[j + half]);
-    const float y = dim < half ? (x0 * c - x1 * s) : (x0 * s + x1 * c);
-    __nv_bfloat16 yb = __float2bfloat16_rn(y);
-    dst[(size_t)h * a.n_out] = *reinterpret_cast<uint16_t*>(&yb);
+    const uint16_t* src = a.src + ((size_t)tok * a.heads + h) * a.d;
+    uint16_t* dst = a.dst + ((size_t)tok * a.heads + h) * a.n_out;
+    float x0[8], x1[8], y0[8], y1[8];
+    unpack8(*reinterpret_cast<const uint4*>(src + j0), x0);
+    unpack8(*reinterpret_cast<const uint4*>(src + j0 + half), x1);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      y0[e] = x0[e] * c[e] - x1[e] * s[e];
+      y1[e] = x0[e] * s[e] + x1[e] * c[e];
+    }
+    if (col0 >= 0) *reinterpret_cast<uint4*>(dst + col0) = pack8(y0);
+    if (col1 >= 0) *reinterpret_cast<uint4*>(dst + col1) = pack8(y1);
+    if (pad)
+      for (int z = a.d; z < 64; z += 8) *reinterpret_cast<uint4*>(dst + z) = make_uint4(0, 0, 0, 0);
   }
 }
 
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream) {
-  const long long total = (long long)a.tokens * a.n_out;
-  if (total == 0) return cudaSuccess;
-  const int threads = 256;
+  const long long total = (long long)a.tokens * (a.d / 16);
+  if (total == 0 || a.n_out == 0) return cudaSuccess;
+  const int threads = 128;
   const long long blocks = (total + threads - 1) / threads;
   rope_side_kernel<<<(unsigned)blocks, threads, 0, stream>>>(a);
   return cudaGetLastError();
