@@ -244,20 +244,20 @@ int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch,
   if (batch < 1 || n_q < 1 || max_cache_len < 0 || !num_splits) return GEMMA_ATTN_ERR_INVALID_ARG;
   int keys = params->kind == GEMMA_ATTN_LOCAL ? std::min(max_cache_len, params->window) : max_cache_len;
   keys += n_q;
-  // One decode CTA per SM at a time: pick the split count whose CTA total fills whole
-  // waves of 148 best, with at least two waves' worth of CTAs where the keys allow and
-  // at least 512 keys (8 chunks) per split.
+  // One decode CTA per SM at a time. Splits run in waves of 148 CTAs, and each CTA
+  // pays a fixed cost (angle tables, the first copies' latency, the merge) worth about
+  // kSplitOverheadKeys keys of streaming: take the split count with the least
+  // waves * (keys per split + that overhead), at least 256 keys per split.
+  constexpr int kSplitOverheadKeys = 512;
   const int sms = 148;
-  const int units = batch * params->num_kv_heads;
-  const int s_cap = std::max(1, keys / 512);
-  const int s_min = std::min(s_cap, std::max(1, (2 * sms + units - 1) / units));
-  int best = s_min;
-  double best_eff = 0.0;
-  for (int s = s_min; s <= std::min(s_cap, 4 * s_min); ++s) {
-    const long long ctas = (long long)units * s;
-    const long long waves = (ctas + sms - 1) / sms;
-    const double eff = (double)ctas / (double)(waves * sms);
-    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+  const long long units = (long long)batch * params->num_kv_heads;
+  const int s_cap = std::max(1, std::min(keys / 256, 4096));
+  int best = 1;
+  double best_cost = 0.0;
+  for (int s = 1; s <= s_cap; ++s) {
+    const long long waves = (units * s + sms - 1) / sms;
+    const double cost = (double)waves * ((double)((keys + s - 1) / s) + kSplitOverheadKeys);
+    if (s == 1 || cost < best_cost * (1.0 - 1e-9)) { best_cost = cost; best = s; }
   }
   *num_splits = best;
   return GEMMA_ATTN_OK;
@@ -299,6 +299,7 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   a.r = rotated_pairs(params->rope_p, params->head_dim);
   a.log2_base = log2((double)params->rope_base);
   a.softmax_scale = params->softmax_scale;
+  if (!decode_supported(a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   if (launch_decode(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
   t_launches = 1;
   return GEMMA_ATTN_OK;

@@ -31,6 +31,7 @@ constexpr int kDecThreads = 128;
 constexpr int kDecWarps = 4;
 constexpr int kCK = 64;  // keys per chunk
 
+constexpr size_t kMaxSmem = 227 * 1024;  // dynamic shared memory one CTA may hold
 constexpr int kDecHeader = 128;  // bytes at the start of shared memory: two mbarriers, abort flag
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -125,7 +126,7 @@ decode_tc_kernel(DecodeArgs a) {
     for (int s = 0; s < NKS; ++s)
       if (s * 16 < r || (s * 16 < HALF + r && s * 16 + 16 > HALF)) rot_bits |= 1u << s;
 
-  extern __shared__ __align__(16) uint8_t dsm[];
+  extern __shared__ __align__(128) uint8_t dsm[];
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(dsm);          // [2], one per chunk buffer
   volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + 16);
   uint16_t* kbuf = reinterpret_cast<uint16_t*>(dsm + kDecHeader);
@@ -495,7 +496,7 @@ static cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
     for (int s = 0; s < D / 16; ++s)
       if (s * 16 < a.r || (s * 16 < D / 2 + a.r && s * 16 + 16 > D / 2)) ++nrk;
   const size_t smem = dec_smem_bytes<D, NT>(!kv_same, nrk);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  if (smem > kMaxSmem) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -504,19 +505,513 @@ static cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Warp-independent decode for up to 8 query rows per (sequence, KV head): plain decode
+// (n_q = 1) and short verify. Each of the NW warps (8, or 4 where 8 do not fit) streams its
+// own 16-key blocks (blocks w, w + NW, ... of the split) through a private ring (one or two
+// stages) of per-row bulk copies
+// and runs the whole block itself:
+//   1. the p-RoPE rotation of the block's keys: each lane takes two pairs, computes
+//      the exact angle of the block's first key and steps it by theta_j per key;
+//   2. S^T = K Q^T with mma.sync (keys on M, query rows on N);
+//   3. mask and online softmax in registers, with the running maximum raised only when
+//      a block's maximum exceeds it by more than 2^8;
+//   4. P^T becomes the B operand of the value product by an 8x8 transpose (movmatrix)
+//      of the packed score fragments, and O^T over the whole head dim accumulates in
+//      registers.
+// No barrier joins the warps until their partial states are merged at the end.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kWB = 16;        // keys per warp block
+// header: mbarriers [warps][stages] at 0, abort flag at 128, merge maxima [warps][8]
+// at 256 and sums [warps][8] after them
+constexpr int kWMgM = 256;
+__host__ __device__ constexpr int wmg_l(int nw) { return kWMgM + nw * 32; }
+__host__ __device__ constexpr int wheader(int nw) { return (wmg_l(nw) + nw * 32 + 127) / 128 * 128; }
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
+
+// Shared-memory carve-up of decode_warp_kernel<D, NS, NW>; r is the rotated pair count and nrk
+// the number of rotated 16-dim k-steps kept in the per-warp rotated copy (K=V layers).
+template <int D, int NS, int NW>
+struct DecWLayout {
+  static constexpr int KST = D + 8;  // bf16 row stride of key / value / query rows
+  static constexpr int RED = D + 4;  // fp32 row stride of the merge buffer
+  size_t qs, stp, bstp, itf, regions, region, k_off, v_off, rot_off, ast_off, total;
+  int rr2, rst;
+  __host__ __device__ DecWLayout(bool kv_same, int r, int nrk) {
+    // table length: even, past r, and covering every word the rotation pass visits
+    rr2 = (r + 2) & ~1;
+    if (kv_same && 16 * ((r + 15) / 16) > rr2) rr2 = 16 * ((r + 15) / 16);
+    rst = nrk * 16 + 8;
+    qs = wheader(NW);
+    stp = qs + align128((size_t)8 * KST * 2);
+    bstp = stp + align128((size_t)rr2 * 8);
+    itf = bstp + align128((size_t)rr2 * 8);
+    regions = itf + align128((size_t)rr2 * 8);
+    k_off = 0;
+    v_off = (size_t)NS * kWB * KST * 2;
+    rot_off = kv_same ? v_off : 2 * v_off;
+    ast_off = rot_off + (kv_same ? (size_t)kWB * rst * 2 : 0);
+    const int nwords = kv_same ? 8 * ((r + 15) / 16) : (r + 1) / 2;
+    region = align128(ast_off + (size_t)(nwords > 0 ? nwords : 1) * 16);
+    const size_t merge = (size_t)NW * 8 * RED * 4;  // the merge buffer reuses the regions
+    total = regions + (NW * region > merge ? NW * region : merge);
+  }
+};
+
+__host__ __device__ inline bool rotated_kstep(int s, int half, int r) {
+  return s * 16 < r || (s * 16 < half + r && s * 16 + 16 > half);
+}
+
+}  // namespace
+
+template <int D, int NS, int NW>
+__global__ void __launch_bounds__(NW * 32)
+decode_warp_kernel(DecodeArgs a) {
+  using L = DecWLayout<D, NS, NW>;
+  constexpr int kWWarps = NW;
+  constexpr int kWStages = NS;  // ring stages per warp
+  constexpr int HALF = D / 2;
+  constexpr int KST = L::KST;
+  constexpr int NKS = D / 16;
+  constexpr bool kQReg = D <= 256;  // query fragments held in registers
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int group = a.num_q_heads / a.num_kv_heads;
+  const int R = group * a.n_q;  // <= 8
+  const bool kv_same = a.v_cache == nullptr;
+  const int len = a.cache_seqlens[b];
+  const int first = a.is_local ? max(0, len - a.window + 1) : 0;  // oldest position any query sees
+  const int nk = (len - first) + a.n_q;
+  const int per = (nk + a.num_splits - 1) / a.num_splits;
+  const int v_lo = min(nk, split * per);
+  const int v_hi = min(nk, v_lo + per);
+  const int r = a.r;
+  const int c16 = (r + 15) / 16;  // rotated k-steps in each half of the head dim
+  uint32_t rot_bits = 0;          // bit s: k-step s of the scores reads the rotated copy
+  int nrk = 0;
+  if (kv_same)
+    for (int s = 0; s < NKS; ++s)
+      if (rotated_kstep(s, HALF, r)) { rot_bits |= 1u << s; ++nrk; }
+  const L lay(kv_same, r, nrk);
+  const int RST = lay.rst;
+
+  extern __shared__ __align__(128) uint8_t dsm[];
+  static_assert(kWWarps * NS * 8 <= 128, "mbarriers overflow their header slot");
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm);  // [warps][stages]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + 128);
+  float* mg_m = reinterpret_cast<float*>(dsm + kWMgM);  // [warps][8]
+  float* mg_l = reinterpret_cast<float*>(dsm + wmg_l(NW));  // [warps][8]
+  uint16_t* qs = reinterpret_cast<uint16_t*>(dsm + lay.qs);
+  float2* stp = reinterpret_cast<float2*>(dsm + lay.stp);
+  float2* bstp = reinterpret_cast<float2*>(dsm + lay.bstp);
+  double* itf = reinterpret_cast<double*>(dsm + lay.itf);
+  uint8_t* region = dsm + lay.regions + (size_t)warp * lay.region;
+  uint16_t* kst = reinterpret_cast<uint16_t*>(region + lay.k_off);
+  uint16_t* vst = reinterpret_cast<uint16_t*>(region + lay.v_off);
+  uint16_t* rbuf = reinterpret_cast<uint16_t*>(region + lay.rot_off);
+  float4* ast = reinterpret_cast<float4*>(region + lay.ast_off);  // this warp's block anchors
+  uint64_t* wbar = bars + warp * kWStages;
+
+  // blocks of this warp: warp, warp + NW, ... of the split's ceil((v_hi - v_lo) / 16)
+  const int nblk = (v_hi - v_lo + kWB - 1) / kWB;
+  const int my_n = nblk > warp ? (nblk - warp + kWWarps - 1) / kWWarps : 0;
+
+  // Bulk copies of block `itx` of this warp into stage itx % 2: lanes 0..15 copy key
+  // rows, lanes 16..31 value rows (separate-V layers); rows past the split are not read.
+  auto issue = [&](int itx) {
+    const int st = itx % kWStages;
+    const int v0 = v_lo + (warp + kWWarps * itx) * kWB;
+    const int nvalid = min(kWB, v_hi - v0);
+    fence_proxy_async_smem();  // earlier generic accesses to this stage come first
+    if (lane == 0) mbar_arrive_expect_tx(&wbar[st], (uint32_t)(nvalid * D * 2 * (kv_same ? 1 : 2)));
+    __syncwarp();
+    const int row = lane & 15;
+    const bool is_v = lane >= 16;
+    if (row < nvalid && (!is_v || !kv_same)) {
+      const int pos = first + v0 + row;
+      const uint16_t* src;
+      if (pos < len) {
+        const size_t slot = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
+        src = (is_v ? a.v_cache : a.k_cache) + (((size_t)b * a.num_kv_heads + kvh) * a.capacity + slot) * D;
+      } else {
+        src = (is_v ? a.new_v : a.new_k) + (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
+      }
+      uint16_t* dst = (is_v ? vst : kst) + (st * kWB + row) * KST;
+      bulk_load(dst, src, D * 2, &wbar[st]);
+    }
+  };
+
+  if (lane == 0) {
+    for (int s = 0; s < kWStages; ++s) mbar_init(&wbar[s], 1);
+    fence_barrier_init();
+  }
+  if (tid == 0) *abort_flag = 0;
+  __syncwarp();
+  // the first blocks stream in while the CTA prepares queries and angle tables
+  for (int s = 0; s < kWStages && s < my_n; ++s) issue(s);
+
+  // rotated queries (bf16); rows R..7 are zero
+  for (int idx = tid; idx < 8 * HALF; idx += kWWarps * 32) {
+    const int row = idx / HALF, j = idx % HALF;
+    float y0 = 0.f, y1 = 0.f;
+    if (row < R) {
+      const int i = row / group, hh = row % group;
+      const uint16_t* qrow = a.q + (((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh) * D;
+      const float x0 = bf2f(qrow[j]), x1 = bf2f(qrow[j + HALF]);
+      y0 = x0; y1 = x1;
+      if (j < r) {
+        float c, s;
+        rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
+        y0 = x0 * c - x1 * s;
+        y1 = x0 * s + x1 * c;
+      }
+    }
+    qs[row * KST + j] = f2bf(y0);
+    qs[row * KST + j + HALF] = f2bf(y1);
+  }
+  // per-pair frequencies (turns per position), cos / sin of theta_j (one key) and of
+  // 16 NW theta_j (one block step of a warp); pairs past r get the identity
+  for (int j = tid; j < lay.rr2; j += kWWarps * 32) {
+    const double f = j < r ? rope_inv_freq_turns(j, D, a.log2_base) : 0.0;
+    float c, s;
+    rope_cos_sin(1.0, f, &c, &s);
+    itf[j] = f;
+    stp[j] = make_float2(c, s);
+    rope_cos_sin((double)(kWWarps * kWB), f, &c, &s);
+    bstp[j] = make_float2(c, s);
+  }
+  __syncthreads();
+
+  uint32_t qf[kQReg ? NKS : 1][2];
+  const uint32_t qbase = smem_u32(qs + (lane & 7) * KST + ((lane >> 3) & 1) * 8);
+  if constexpr (kQReg) {
+#pragma unroll
+    for (int s = 0; s < NKS; ++s) ldsm_x2(qbase + s * 32, qf[s][0], qf[s][1]);
+  }
+
+  // per-thread rows 2t and 2t + 1: validity and the query position they belong to
+  bool row_ok[2];
+  int qpos[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int row = 2 * t + e;
+    row_ok[e] = row < R;
+    qpos[e] = len + (row < R ? row / group : 0);
+  }
+  const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  float oacc[NKS][4];
+#pragma unroll
+  for (int mt = 0; mt < NKS; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
+
+  // rotation work: words of two dims; K=V layers copy every word of the rotated
+  // k-steps into the rotated buffer, separate-V layers rotate in place
+  const int nwords = kv_same ? 8 * c16 : (r + 1) / 2;
+  const uint32_t kfrag = (uint32_t)((lane & 15) * KST + (lane >> 4) * 8) * 2;
+  const uint32_t rfrag = (uint32_t)((lane & 15) * RST + (lane >> 4) * 8) * 2;
+  const uint32_t vfrag = (uint32_t)(((lane & 7) + ((lane >> 4) << 3)) * KST + ((lane >> 3) & 1) * 8) * 2;
+
+  int it = 0;
+  bool ok = true;
+  for (; it < my_n; ++it) {
+    const int st = it % kWStages;
+    ok = mbar_wait(&wbar[st], (uint32_t)(it / kWStages) & 1u, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    uint16_t* kd = kst + st * kWB * KST;
+    uint16_t* vdw = kv_same ? kd : vst + st * kWB * KST;
+    const int v0 = v_lo + (warp + kWWarps * it) * kWB;
+    const int nvalid = min(kWB, v_hi - v0);
+    const int pos0 = first + v0;
+    if (nvalid < kWB) {  // value rows past the split end: zero, so that P = 0 meets finite values
+      for (int idx = lane; idx < (kWB - nvalid) * (D / 8); idx += 32) {
+        const int row = nvalid + idx / (D / 8), c8 = idx % (D / 8);
+        *reinterpret_cast<uint4*>(vdw + row * KST + c8 * 8) = make_uint4(0, 0, 0, 0);
+      }
+    }
+
+    // ---- 1. rotation: each lane owns words (pairs j, j + 1) and walks the block's 16
+    // keys from the angle of the block's first key, stepping by theta_j per key. That
+    // anchor angle is exact every 16th block and otherwise the previous block's anchor
+    // advanced by 16 NW theta_j (the warp's stride); all loads come first.
+    if (r > 0) {
+      uint16_t* dst0 = kv_same ? rbuf : kd;
+      const int dst_hi = kv_same ? 16 * c16 : HALF;
+      const int dst_st = kv_same ? RST : KST;
+      const bool exact = (it & 15) == 0;
+      for (int w = lane; w < nwords; w += 32) {
+        const int j = 2 * w;
+        uint32_t w0[kWB], w1[kWB];
+#pragma unroll
+        for (int u = 0; u < kWB; ++u) {
+          w0[u] = *reinterpret_cast<const uint32_t*>(kd + u * KST + j);
+          w1[u] = *reinterpret_cast<const uint32_t*>(kd + u * KST + HALF + j);
+        }
+        float4 an;
+        if (exact) {
+          rope_cos_sin((double)pos0, itf[j], &an.x, &an.y);
+          rope_cos_sin((double)pos0, itf[j + 1], &an.z, &an.w);
+        } else {
+          const float4 pa = ast[w];
+          const float4 bs = *reinterpret_cast<const float4*>(bstp + j);
+          an = make_float4(pa.x * bs.x - pa.y * bs.y, pa.x * bs.y + pa.y * bs.x,
+                           pa.z * bs.z - pa.w * bs.w, pa.z * bs.w + pa.w * bs.z);
+        }
+        ast[w] = an;
+        const float4 st = *reinterpret_cast<const float4*>(stp + j);
+        float ac[2] = {an.x, an.z}, as[2] = {an.y, an.w};
+        const float sc[2] = {st.x, st.z}, ss[2] = {st.y, st.w};
+#pragma unroll
+        for (int u = 0; u < kWB; ++u) {
+          const float x00 = __uint_as_float(w0[u] << 16), x01 = __uint_as_float(w0[u] & 0xFFFF0000u);
+          const float x10 = __uint_as_float(w1[u] << 16), x11 = __uint_as_float(w1[u] & 0xFFFF0000u);
+          const uint32_t o0 = pack_bf16x2(x00 * ac[0] - x10 * as[0], x01 * ac[1] - x11 * as[1]);
+          const uint32_t o1 = pack_bf16x2(x00 * as[0] + x10 * ac[0], x01 * as[1] + x11 * ac[1]);
+          *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + j) = o0;
+          *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + dst_hi + j) = o1;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float nc = ac[e] * sc[e] - as[e] * ss[e];
+            as[e] = ac[e] * ss[e] + as[e] * sc[e];
+            ac[e] = nc;
+          }
+        }
+      }
+    }
+    __syncwarp();
+
+    // ---- 2. S^T = K Q^T for the block's 16 keys (four accumulator chains)
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      float sch[3][4] = {};
+      const uint32_t kbase = smem_u32(kd) + kfrag;
+      const uint32_t rbase = smem_u32(rbuf) + rfrag;
+#pragma unroll
+      for (int s = 0; s < NKS; ++s) {
+        const bool rot = (rot_bits >> s) & 1u;
+        const int slot = __popc(rot_bits & ((1u << s) - 1u));
+        uint32_t a0, a1, a2, a3, b0, b1;
+        ldsm_x4(rot ? rbase + slot * 32 : kbase + s * 32, a0, a1, a2, a3);
+        if constexpr (kQReg) {
+          b0 = qf[s][0];
+          b1 = qf[s][1];
+        } else {
+          ldsm_x2(qbase + s * 32, b0, b1);
+        }
+        mma_16816((s & 3) ? sch[(s & 3) - 1] : sacc, a0, a1, a2, a3, b0, b1);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[e] += (sch[0][e] + sch[1][e]) + sch[2][e];
+    }
+
+    // ---- 3. mask and online softmax; fragment element e: key g + 8 * (e >> 1), row 2t + (e & 1)
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int v = v0 + g + 8 * (e >> 1);
+      const int pos = first + v;
+      const int h = e & 1;
+      const bool vis = row_ok[h] && v < v_hi && pos <= qpos[h] && (!a.is_local || pos > qpos[h] - a.window);
+      sacc[e] = vis ? sacc[e] * scale_log2 : -INFINITY;
+      mx[h] = fmaxf(mx[h], sacc[e]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+    }
+    // the running maximum moves only when a row's block maximum passes it by more than
+    // 8 (log2 units), so P stays below 2^8; the decision is warp-uniform
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + 8.f || mx[1] > m_run[1] + 8.f)) {
+      float al[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float mn = fmaxf(m_run[h], mx[h]);
+        al[h] = mn == -INFINITY ? 1.f : exp2f(m_run[h] - mn);
+        m_run[h] = mn;
+        l_run[h] *= al[h];
+      }
+#pragma unroll
+      for (int mt = 0; mt < NKS; ++mt) {
+        oacc[mt][0] *= al[0];
+        oacc[mt][1] *= al[1];
+        oacc[mt][2] *= al[0];
+        oacc[mt][3] *= al[1];
+      }
+    }
+    const float msub[2] = {m_run[0] == -INFINITY ? 0.f : m_run[0], m_run[1] == -INFINITY ? 0.f : m_run[1]};
+    const uint32_t p01 = pack_bf16x2(exp2f(sacc[0] - msub[0]), exp2f(sacc[1] - msub[1]));  // key g
+    const uint32_t p23 = pack_bf16x2(exp2f(sacc[2] - msub[0]), exp2f(sacc[3] - msub[1]));  // key g + 8
+    l_run[0] += __uint_as_float(p01 << 16) + __uint_as_float(p23 << 16);
+    l_run[1] += __uint_as_float(p01 & 0xFFFF0000u) + __uint_as_float(p23 & 0xFFFF0000u);
+    // P^T B fragment: keys 2t, 2t + 1 (b0) and 2t + 8, 2t + 9 (b1) of query row g
+    const uint32_t pb0 = movmatrix_trans(p01);
+    const uint32_t pb1 = movmatrix_trans(p23);
+
+    // ---- 4. O^T += V^T P^T over the whole head dim
+    {
+      const uint32_t vbase = smem_u32(vdw) + vfrag;
+#pragma unroll
+      for (int mt = 0; mt < NKS; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vbase + mt * 32, a0, a1, a2, a3);
+        mma_16816(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+    }
+    __syncwarp();  // every lane is done with this stage and the rotated copy
+    if (it + kWStages < my_n) issue(it + kWStages);
+  }
+  // Copies still in flight after an early exit land before the warp moves on.
+  if (!ok && lane == 0) {
+    for (int k = it; k < my_n && k < it + kWStages; ++k) {
+      const uint32_t par = (uint32_t)(k / kWStages) & 1u;
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(&wbar[k % kWStages], par) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+    }
+  }
+
+  // ---- merge the warps' (max, sum, O) and write this split's partial
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 4);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
+    if (g == 0) {
+      mg_m[warp * 8 + 2 * t + h] = m_run[h];
+      mg_l[warp * 8 + 2 * t + h] = l_run[h];
+    }
+  }
+  __syncthreads();  // every warp has left its loop: the stage buffers are free
+  auto merged = [&](int row, float& M, float& Lsum) {
+    M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWWarps; ++w) M = fmaxf(M, mg_m[w * 8 + row]);
+    Lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWWarps; ++w) {
+      const float mw = mg_m[w * 8 + row];
+      if (mw != -INFINITY) Lsum += mg_l[w * 8 + row] * exp2f(mw - M);
+    }
+  };
+  float* red = reinterpret_cast<float*>(dsm + lay.regions);  // [warps][8][D + 4]
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float M, Lsum;
+    merged(2 * t + h, M, Lsum);
+    const float f = (Lsum > 0.f && m_run[h] != -INFINITY) ? exp2f(m_run[h] - M) / Lsum : 0.f;
+    float* dst = red + (size_t)(warp * 8 + 2 * t + h) * L::RED + g;
+#pragma unroll
+    for (int mt = 0; mt < NKS; ++mt) {
+      dst[mt * 16] = oacc[mt][h] * f;
+      dst[mt * 16 + 8] = oacc[mt][2 + h] * f;
+    }
+  }
+  __syncthreads();
+  const int rows_total = a.batch * a.n_q * a.num_q_heads;
+  for (int idx = tid; idx < R * D; idx += kWWarps * 32) {
+    const int row = idx / D, d = idx % D;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWWarps; ++w) acc += red[(size_t)(w * 8 + row) * L::RED + d];
+    const size_t orow = ((size_t)b * a.n_q + row / group) * a.num_q_heads + kvh * group + row % group;
+    a.partial_o[((size_t)split * rows_total + orow) * D + d] = acc;
+  }
+  if (tid < R) {
+    float M, Lsum;
+    merged(tid, M, Lsum);
+    const size_t orow = ((size_t)b * a.n_q + tid / group) * a.num_q_heads + kvh * group + tid % group;
+    a.partial_lse[(size_t)split * rows_total + orow] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY;
+  }
+}
+
+template <int D, int NS, int NW>
+static size_t decode_warp_smem(const DecodeArgs& a) {
+  const bool kv_same = a.v_cache == nullptr;
+  int nrk = 0;
+  if (kv_same)
+    for (int s = 0; s < D / 16; ++s)
+      if (rotated_kstep(s, D / 2, a.r)) ++nrk;
+  return DecWLayout<D, NS, NW>(kv_same, a.r, nrk).total;
+}
+
+template <int D, int NS, int NW>
+static cudaError_t launch_decode_warp(const DecodeArgs& a, cudaStream_t stream) {
+  const size_t smem = decode_warp_smem<D, NS, NW>(a);
+  if (smem > kMaxSmem) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<D, NS, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.num_splits, a.num_kv_heads, a.batch);
+  decode_warp_kernel<D, NS, NW><<<grid, NW * 32, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 // Largest supported query-row count per CTA (group * n_q) for a head dim.
 int decode_max_rows(int head_dim) { return head_dim >= 512 ? 32 : 64; }
 
+// Decode kernel variant for a shape: the warp-independent kernel for up to 8 rows (the
+// first of 8 warps x 2 ring stages, 8 x 1, 4 x 1 that fits), the
+// CTA-wide kernel with 16, 32 or 64 row slots above that; kDecNone when no variant fits
+// in shared memory.
+enum DecodeVariant { kDecNone = 0, kDecWarp8x2, kDecWarp8x1, kDecWarp4x1, kDecTc2, kDecTc4, kDecTc8 };
+
+template <int D>
+static int decode_variant_d(const DecodeArgs& a) {
+  const int R = (a.num_q_heads / a.num_kv_heads) * a.n_q;
+  const bool kv_same = a.v_cache == nullptr;
+  int nrk = 0;
+  if (kv_same)
+    for (int s = 0; s < D / 16; ++s)
+      if (rotated_kstep(s, D / 2, a.r)) ++nrk;
+  if (R <= 8) {
+    if (decode_warp_smem<D, 2, 8>(a) <= kMaxSmem) return kDecWarp8x2;
+    if (decode_warp_smem<D, 1, 8>(a) <= kMaxSmem) return kDecWarp8x1;
+    if (decode_warp_smem<D, 1, 4>(a) <= kMaxSmem) return kDecWarp4x1;
+    return kDecNone;
+  }
+  if (R <= 16) return dec_smem_bytes<D, 2>(!kv_same, nrk) <= kMaxSmem ? kDecTc2 : kDecNone;
+  if (R <= 32) return dec_smem_bytes<D, 4>(!kv_same, nrk) <= kMaxSmem ? kDecTc4 : kDecNone;
+  if (R <= 64 && D < 512) return dec_smem_bytes<D, 8>(!kv_same, nrk) <= kMaxSmem ? kDecTc8 : kDecNone;
+  return kDecNone;
+}
+
 template <int D>
 static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t stream) {
-  const int R = (a.num_q_heads / a.num_kv_heads) * a.n_q;
-  if (R <= 8) return launch_decode_tc<D, 1>(a, stream);
-  if (R <= 16) return launch_decode_tc<D, 2>(a, stream);
-  if (R <= 32) return launch_decode_tc<D, 4>(a, stream);
-  if constexpr (D < 512) {
-    if (R <= 64) return launch_decode_tc<D, 8>(a, stream);
+  switch (decode_variant_d<D>(a)) {
+    case kDecWarp8x2: return launch_decode_warp<D, 2, 8>(a, stream);
+    case kDecWarp8x1: return launch_decode_warp<D, 1, 8>(a, stream);
+    case kDecWarp4x1: return launch_decode_warp<D, 1, 4>(a, stream);
+    case kDecTc2: return launch_decode_tc<D, 2>(a, stream);
+    case kDecTc4: return launch_decode_tc<D, 4>(a, stream);
+    case kDecTc8:
+      if constexpr (D < 512) return launch_decode_tc<D, 8>(a, stream);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
   }
-  return cudaErrorInvalidValue;
+}
+
+bool decode_supported(const DecodeArgs& a) {
+  switch (a.head_dim) {
+    case 32: return decode_variant_d<32>(a) != kDecNone;
+    case 64: return decode_variant_d<64>(a) != kDecNone;
+    case 128: return decode_variant_d<128>(a) != kDecNone;
+    case 256: return decode_variant_d<256>(a) != kDecNone;
+    case 512: return decode_variant_d<512>(a) != kDecNone;
+    default: return false;
+  }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
@@ -533,43 +1028,38 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 // ---------------------------------------------------------------------------
 // Combine: one warp per output row.
 // ---------------------------------------------------------------------------
+// One thread per output element (row, dim): the row's split weights exp(lse_s - max)
+// are recomputed by every thread of the row (the split log-sum-exps stay in L1), and
+// the partial reads are coalesced across the threads of a row.
 __global__ void combine_kernel(CombineArgs a) {
-  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= a.rows) return;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.rows * a.head_dim) return;
+  const int row = (int)(idx / a.head_dim), c = (int)(idx % a.head_dim);
   float mm = -INFINITY;
-  for (int s = lane; s < a.num_splits; s += 32) mm = fmaxf(mm, a.partial_lse[(size_t)s * a.rows + row]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
-  float den = 0.f;
-  for (int s = lane; s < a.num_splits; s += 32) {
-    const float l = a.partial_lse[(size_t)s * a.rows + row];
-    if (l != -INFINITY) den += __expf(l - mm);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  for (int c = lane; c < a.head_dim; c += 32) {
-    float acc = 0.f;
-    if (mm != -INFINITY) {
-      for (int s = 0; s < a.num_splits; ++s) {
-        const float l = a.partial_lse[(size_t)s * a.rows + row];
-        if (l == -INFINITY) continue;
-        acc += __expf(l - mm) * a.partial_o[((size_t)s * a.rows + row) * a.head_dim + c];
-      }
-      acc /= den;
+  for (int s = 0; s < a.num_splits; ++s) mm = fmaxf(mm, a.partial_lse[(size_t)s * a.rows + row]);
+  float den = 0.f, acc = 0.f;
+  if (mm != -INFINITY) {
+    for (int s = 0; s < a.num_splits; ++s) {
+      const float l = a.partial_lse[(size_t)s * a.rows + row];
+      if (l == -INFINITY) continue;
+      const float w = __expf(l - mm);
+      den += w;
+      acc += w * a.partial_o[((size_t)s * a.rows + row) * a.head_dim + c];
     }
-    if (a.out_f32)
-      reinterpret_cast<float*>(a.out)[(size_t)row * a.head_dim + c] = acc;
-    else
-      reinterpret_cast<__nv_bfloat16*>(a.out)[(size_t)row * a.head_dim + c] = __float2bfloat16_rn(acc);
+    acc /= den;
   }
-  if (lane == 0 && a.lse != nullptr) a.lse[row] = (mm == -INFINITY) ? -INFINITY : mm + logf(den);
+  if (a.out_f32)
+    reinterpret_cast<float*>(a.out)[idx] = acc;
+  else
+    reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(acc);
+  if (c == 0 && a.lse != nullptr) a.lse[row] = (mm == -INFINITY) ? -INFINITY : mm + logf(den);
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
-  if (a.rows == 0) return cudaSuccess;
-  const int warps = 8;
-  combine_kernel<<<(a.rows + warps - 1) / warps, warps * 32, 0, stream>>>(a);
+  const long long total = (long long)a.rows * a.head_dim;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  combine_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

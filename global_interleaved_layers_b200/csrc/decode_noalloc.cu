@@ -118,6 +118,7 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   a.r = rotated_pairs(params->rope_p, d);
   a.log2_base = log2((double)params->rope_base);
   a.softmax_scale = params->softmax_scale;
+  if (!decode_supported(a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (launch_decode(a, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
 

@@ -66,6 +66,7 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 int decode_max_rows(int head_dim);  // largest group * n_q one decode CTA handles
+bool decode_supported(const DecodeArgs& a);  // a kernel variant fits this shape
 
 struct CombineArgs {
   const float* partial_o;

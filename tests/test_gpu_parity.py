@@ -206,6 +206,23 @@ def test_decode_global_gqa8():
     _check_decode(W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6), (1500,), 1, G.CACHE_CONTIGUOUS)
 
 
+@pytest.mark.parametrize("kind,hq,hkv,d,p,n_q", [
+    (W.GLOBAL, 4, 1, 32, 1.0, 1),     # r = 16: every k-step rotated
+    (W.GLOBAL, 2, 1, 64, 0.5, 3),     # r = 16
+    (W.GLOBAL, 8, 2, 128, 0.3, 1),    # r = 19: odd, rotated k-steps partly pass-through
+    (W.GLOBAL, 4, 1, 256, 0.1, 2),    # r = 12
+    (W.LOCAL, 4, 2, 32, 1.0, 2),
+    (W.LOCAL, 8, 4, 64, 0.75, 4),     # r = 24
+    (W.LOCAL, 2, 2, 128, 0.3, 1),     # r = 19
+    (W.LOCAL, 8, 1, 512, 1.0, 1),     # separate-V d = 512: one ring stage per warp
+])
+def test_decode_head_dims_and_partial_rotation(kind, hq, hkv, d, p, n_q):
+    window = 48 if kind == W.LOCAL else 0
+    layer = W.LayerSpec(kind, hq, hkv, d, window=window, rope_p=p, rope_base=1e4)
+    layout = G.CACHE_RING if kind == W.LOCAL else G.CACHE_CONTIGUOUS
+    _check_decode(layer, (0, 37, 130), n_q, layout, 3)
+
+
 def test_combine_against_oracle():
     rng = np.random.default_rng(9)
     S, R, d = 5, 37, 64
