@@ -362,7 +362,7 @@ int gemma_attn_check(void* stream_) {
 
 int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const void* p, float* d, void* stream_) {
   t_launches = 0;
-  if ((mode != 0 && mode != 1) || !b || !d || (mode == 0 && !a) || (mode == 1 && !p))
+  if (mode < 0 || mode > 2 || !b || !d || (mode == 0 && !a) || (mode != 0 && !p))
     return GEMMA_ATTN_ERR_INVALID_ARG;
   CUtensorMap am, bm;
   bool ok = true;
@@ -370,7 +370,7 @@ int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const v
     ok &= make_map(&am, a, 128, 1, 128, 128);
     ok &= make_map(&bm, b, 128, 1, 128, 128);
   } else {
-    ok &= make_map(&bm, b, 64, 1, 128, 128);
+    ok &= make_map(&bm, b, mode == 1 ? 64 : 128, 1, 128, 128);
     am = bm;
   }
   if (!ok) return GEMMA_ATTN_ERR_LAUNCH;

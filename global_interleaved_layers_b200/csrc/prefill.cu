@@ -42,7 +42,8 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kChunk = 64;                   // dims per TMA box / swizzle row
-constexpr int kStageBytes = 16384;           // one ring stage
+constexpr int kChunkBytes = 16384;           // 128 rows x 64 dims of bf16: a Q chunk or a V chunk
+constexpr int kMaxStages = 16;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
@@ -54,17 +55,27 @@ struct PrefillCfg {
   static constexpr int kSplit = D / kDv;                      // work units per (tile, head)
   static constexpr int kQChunks = D / kChunk;
   static constexpr int kVChunks = kDv / kChunk;
-  static constexpr int kQBytes = kQChunks * kStageBytes;
-  static constexpr int kStages = D >= 512 ? 6 : 8;
-  // Single CTA: a K stage is one 64-dim chunk of 128 keys; a V stage one 64-dim chunk.
-  // Pair: a K stage is two 64-dim chunks of this CTA's 64 keys; a V stage one 64-dim
-  // chunk of 128 keys (the pair's two CTAs hold adjacent chunks).
-  static constexpr int kKStages = PAIR ? kQChunks / 2 : kQChunks;
-  static constexpr int kVStages = PAIR ? kVChunks / 2 : kVChunks;
+  static constexpr int kQBytes = kQChunks * kChunkBytes;
+  // Ring stages. Single CTA: 16 KB, a K stage is one 64-dim chunk of 128 keys and a V
+  // stage one 64-column chunk. Pair with d >= 256: 32 KB, a K stage is four 64-dim chunks
+  // of this CTA's 64 keys and a V stage two 64-column chunks of 128 keys (the pair's CTAs
+  // hold adjacent column pairs, so one PV MMA is N = 256). Pair with d = 128: 16 KB, two
+  // K chunks or one V chunk. Fewer, larger stages mean fewer barrier round trips per tile.
+  static constexpr int kStageBytes = (PAIR && D >= 256) ? 2 * kChunkBytes : kChunkBytes;
+  static constexpr int kKChunkBytes = PAIR ? kChunkBytes / 2 : kChunkBytes;
+  static constexpr int kKPerStage = kStageBytes / kKChunkBytes;
+  static constexpr int kVPerStage = kStageBytes / kChunkBytes;
+  static constexpr int kKStages = kQChunks / kKPerStage;
+  static constexpr int kVStages = (PAIR ? kVChunks / 2 : kVChunks) / kVPerStage;
+  static constexpr int kPvN = (PAIR ? 2 : 1) * kVPerStage * kChunk;  // output columns per V stage
+  static constexpr int kRingBudget = 232448 - 1024 /*align*/ - 512 /*barriers*/ - kQBytes;
+  static constexpr int kStages = kRingBudget / kStageBytes < kMaxStages ? kRingBudget / kStageBytes : kMaxStages;
   static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
   static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(!PAIR || D >= 128, "paired form needs at least two 64-dim chunks");
+  static_assert(kKStages >= 1 && kVStages >= 1 && kStages >= 2, "ring shape");
+  static_assert(kPvN <= 256, "PV MMA width");
 };
 
 struct __align__(8) Barriers {
@@ -72,14 +83,21 @@ struct __align__(8) Barriers {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done;
+  uint64_t o_ready;  // one phase: every PV of the work unit has finished
   uint64_t mma_done;
-  uint64_t ring_full[8];
-  uint64_t ring_empty[8];
+  uint64_t ring_full[kMaxStages];
+  uint64_t ring_empty[kMaxStages];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+// 2^x on the SFU (ex2.approx, flush-to-zero): P is rounded to bf16 and the row sums
+// carry far more error than the approximation's few ulp.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Waits that may be satisfied by the other CTA of a pair use cluster-scope acquire.
 template <bool PAIR>
@@ -135,9 +153,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     mbar_init(&bars->q_full, load_arrivals);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], PAIR ? 256 : 128);
+      mbar_init(&bars->p_full[b], PAIR ? 8 : 4);  // one arrival per softmax warp (of both CTAs)
     }
     mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->o_ready, 1);
     mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&bars->ring_full[s], load_arrivals);
@@ -185,8 +204,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
 
       expect(&bars->q_full, Cfg::kQBytes);
       for (int c = 0; c < Cfg::kQChunks; ++c) {
-        if ((args.rot_mask >> c) & 1) load(q_smem + c * kStageBytes, &qs_map, &bars->q_full, rot_idx(c) * kChunk, head, tok0 + row0);
-        else load(q_smem + c * kStageBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
+        if ((args.rot_mask >> c) & 1) load(q_smem + c * kChunkBytes, &qs_map, &bars->q_full, rot_idx(c) * kChunk, head, tok0 + row0);
+        else load(q_smem + c * kChunkBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
       }
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
@@ -197,16 +216,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           for (int s = 0; s < Cfg::kKStages && ok; ++s) {
             ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
             if (!ok) break;
-            expect(&bars->ring_full[st], kStageBytes);
-            uint8_t* dst = ring + st * kStageBytes;
+            expect(&bars->ring_full[st], Cfg::kStageBytes);
+            uint8_t* dst = ring + st * Cfg::kStageBytes;
             if constexpr (PAIR) {
-              // chunks 2s and 2s+1 of this CTA's 64 keys
-              for (int sub = 0; sub < 2; ++sub) {
-                const int c = 2 * s + sub;
+              // chunks kKPerStage * s + sub of this CTA's 64 keys
+              for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
+                const int c = Cfg::kKPerStage * s + sub;
                 if ((args.rot_mask >> c) & 1)
-                  load(dst + sub * 8192, &ks64_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh, key0 + 64 * (int)rank);
+                  load(dst + sub * Cfg::kKChunkBytes, &ks64_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh,
+                       key0 + 64 * (int)rank);
                 else
-                  load(dst + sub * 8192, &k64_map, &bars->ring_full[st], c * kChunk, kvh, key0 + 64 * (int)rank);
+                  load(dst + sub * Cfg::kKChunkBytes, &k64_map, &bars->ring_full[st], c * kChunk, kvh,
+                       key0 + 64 * (int)rank);
               }
             } else {
               const int c = s;
@@ -221,9 +242,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           for (int s = 0; s < Cfg::kVStages && ok; ++s) {
             ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
             if (!ok) break;
-            expect(&bars->ring_full[st], kStageBytes);
-            const int c = PAIR ? 2 * s + (int)rank : s;
-            load(ring + st * kStageBytes, &v_map, &bars->ring_full[st], vpart * Cfg::kDv + c * kChunk, kvh, key0);
+            expect(&bars->ring_full[st], Cfg::kStageBytes);
+            // this CTA's column chunks of V stage s: the pair's two CTAs hold adjacent groups
+            for (int sub = 0; sub < Cfg::kVPerStage; ++sub) {
+              const int c = ((PAIR ? 2 * s + (int)rank : s) * Cfg::kVPerStage) + sub;
+              load(ring + st * Cfg::kStageBytes + sub * kChunkBytes, &v_map, &bars->ring_full[st],
+                   vpart * Cfg::kDv + c * kChunk, kvh, key0);
+            }
             next();
           }
         }
@@ -249,14 +274,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
       constexpr int M = PAIR ? 2 * kBM : kBM;
-      constexpr int PV_N = PAIR ? 2 * kChunk : kChunk;
+      constexpr int PV_N = Cfg::kPvN;
       const uint32_t idesc_qk = umma_idesc_bf16(M, kBN, 0, 0);
       const uint32_t idesc_pv = umma_idesc_bf16(M, PV_N, 0, 1);
       // descriptors of stage 0 / Q chunk 0; other stages and k-steps are offsets of
       // (bytes >> 4) in the low start-address field
       const uint64_t q_desc0 = sdesc_sw128(smem_u32(q_smem), 16, 1024);
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(ring), 16, 1024);
-      const uint64_t v_desc0 = sdesc_sw128(smem_u32(ring), kStageBytes, 1024);
+      // V is MN-major: 64-column chunks of a stage are kChunkBytes apart (leading offset)
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(ring), kChunkBytes, 1024);
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
       bool ok = wait_bar<PAIR>(&bars->q_full, 0, abort_flag);
@@ -270,12 +296,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
             ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t kd = k_desc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint64_t kd = k_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
 #pragma unroll
-            for (int sub = 0; sub < (PAIR ? 2 : 1); ++sub) {
-              const int c = PAIR ? 2 * s + sub : s;
-              const uint64_t qd = q_desc0 + (uint64_t)((c * kStageBytes) >> 4);
-              const uint64_t kds = kd + (uint64_t)((sub * 8192) >> 4);
+            for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
+              const int c = Cfg::kKPerStage * s + sub;
+              const uint64_t qd = q_desc0 + (uint64_t)((c * kChunkBytes) >> 4);
+              const uint64_t kds = kd + (uint64_t)((sub * Cfg::kKChunkBytes) >> 4);
 #pragma unroll
               for (int kk = 0; kk < kChunk / 16; ++kk) {
                 if constexpr (PAIR) umma_ss_pair(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
@@ -301,7 +327,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
             ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t vd = v_desc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint64_t vd = v_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
             const uint32_t o_col = kColO + s * PV_N;
 #pragma unroll
             for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -316,6 +342,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           if constexpr (PAIR) umma_commit_pair_both(&bars->pv_done);
           else umma_commit(&bars->pv_done);
         }
+      }
+      // The epilogue waits on o_ready, a single-phase barrier: softmax warps skip pv_done
+      // phases, so a parity wait on pv_done could not tell the last phase from an older one.
+      if (ok) {
+        if constexpr (PAIR) umma_commit_pair_both(&bars->o_ready);
+        else umma_commit(&bars->o_ready);
       }
       // All MMAs issued by this thread are complete once mma_done fires.
       if constexpr (PAIR) umma_commit_pair_local(&bars->mma_done);
@@ -349,7 +381,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
       const bool partial = (kt + 1) * kBN > len ||
                            kv_tile_class(is_local, args.window, len, qt, kt, kBM, kBN) != kTileFull;
-      float m_tile = -INFINITY;
+      // Masked tiles are scaled here (masked entries -inf); full tiles keep raw scores and
+      // fold the scale into the exponent's FFMA (scale > 0, so the max commutes with it).
+      // Eight partial maxima keep the reduction off one long dependency chain.
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       if (partial) {
         const int k0 = kt * kBN;
 #pragma unroll
@@ -357,15 +394,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           const int key = k0 + c;
           const bool vis = key <= grow && (!is_local || key > grow - args.window);
           t[c] = vis ? t[c] * scale_log2 : -INFINITY;
-          m_tile = fmaxf(m_tile, t[c]);
+          mx8[c & 7] = fmaxf(mx8[c & 7], t[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          t[c] *= scale_log2;
-          m_tile = fmaxf(m_tile, t[c]);
-        }
+        for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], t[c]);
       }
+      const float coef = partial ? 1.f : scale_log2;
+      float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      if (!partial) m_tile *= scale_log2;
       // Raise the running max only when it grows by more than 2^8 (or was empty); P
       // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
       float alpha = 1.f;
@@ -383,19 +421,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       // wait for PV(jj-1), so the exponentials stay off the PV -> softmax -> PV chain.
       const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t p[kBN / 2];
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN / 2; ++c) {
-        float p0 = fast_exp2(t[2 * c] - m_sub);
-        float p1 = fast_exp2(t[2 * c + 1] - m_sub);
-        rs += p0 + p1;
+        const float p0 = fast_exp2(fmaf(t[2 * c], coef, -m_sub));
+        const float p1 = fast_exp2(fmaf(t[2 * c + 1], coef, -m_sub));
+        rs4[c & 3] += p0 + p1;
         p[c] = pack_bf16x2(p0, p1);
       }
-      l_sum += rs;
+      l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_st_x32(tmem + lane_off + s_col, p);
       tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
-      // O may only be touched once PV(jj-1) has finished.
-      if (jj >= 1) {
+      // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
+      // lane needs it, each lane with its own factor (1 for lanes that do not). O may only
+      // be touched once PV(jj-1) has finished; without a rescale the warp does not wait,
+      // since PV(jj) is issued after PV(jj-1) and the tensor core runs them in order.
+      // The parity wait is exact: S(jj) was issued after PV(jj-2) finished, and PV(jj)
+      // needs this warp's p_full(jj) arrival below, so PV(jj-1) is the only pv_done phase
+      // that can still be pending.
+      const bool rescale_warp = __any_sync(0xffffffffu, rescale_o);
+      if (rescale_warp && jj >= 1) {
         ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag));
         if (!ok) {
           tmem_st_wait();  // the P stores land before the teardown frees TMEM
@@ -403,9 +448,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         }
         tc_fence_after();
       }
-      // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
-      // lane needs it, each lane with its own factor (1 for lanes that do not).
-      if (__any_sync(0xffffffffu, rescale_o)) {
+      if (rescale_warp) {
 #pragma unroll 1
         for (int c = 0; c < Cfg::kDv / 32; ++c) {
           uint32_t o[32];
@@ -418,11 +461,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       }
       tmem_st_wait();
       tc_fence_before();
-      if (!PAIR || leader) mbar_arrive(&bars->p_full[b]);
-      else mbar_arrive_cluster(smem_u32(&bars->p_full[b]) & kPeerBitMask);
+      __syncwarp();  // every lane's P and O stores precede the warp's single arrival
+      if (lane == 0) {
+        if (!PAIR || leader) mbar_arrive(&bars->p_full[b]);
+        else mbar_arrive_cluster(smem_u32(&bars->p_full[b]) & kPeerBitMask);
+      }
     }
     if (ok && ntiles > 0)
-      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->o_ready, 0u, abort_flag));
     if (ok) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;

@@ -4,6 +4,9 @@
 //           (two 64-column swizzled chunks each), as for S = Q K^T.
 //   mode 1: D[128x64] = P[128x128] * V[128x64], P written to tensor memory as bf16
 //           pairs by tcgen05.st, V MN-major in shared memory, as for O += P V.
+//   mode 2: D[128x128] = P[128x128] * V[128x128], V as two 64-column MN-major chunks
+//           16 KB apart (the descriptor's leading byte offset), as for a 128-column
+//           share of an N = 256 paired PV product.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -42,11 +45,12 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_con
         tma_load_3d(b_s + c * 16384, &b_map, &bar_load, c * 64, 0, 0);
       }
     } else {
-      mbar_arrive_expect_tx(&bar_load, 16384);
-      tma_load_3d(b_s, &b_map, &bar_load, 0, 0, 0);
+      const int nchunks = mode == 1 ? 1 : 2;
+      mbar_arrive_expect_tx(&bar_load, 16384u * nchunks);
+      for (int c = 0; c < nchunks; ++c) tma_load_3d(b_s + c * 16384, &b_map, &bar_load, c * 64, 0, 0);
     }
   }
-  if (mode == 1) {
+  if (mode != 0) {
     // row `threadIdx.x` of P into TMEM columns [128, 192) as bf16 pairs
     const int row = warp * 32 + lane;
     uint32_t pk[64];
@@ -61,7 +65,7 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_con
   if (threadIdx.x == 0) {
     volatile int* ab = &abort_flag;
     bool ok = mbar_wait(&bar_load, 0, ab);
-    if (ok && mode == 1) ok = mbar_wait(&bar_p, 0, ab);
+    if (ok && mode != 0) ok = mbar_wait(&bar_p, 0, ab);
     tc_fence_after();
     if (ok) {
       if (mode == 0) {
@@ -73,7 +77,7 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_con
             umma_ss(tmem, ad, bd, idesc, (c | kk) != 0);
           }
       } else {
-        const uint32_t idesc = umma_idesc_bf16(128, 64, 0, 1);
+        const uint32_t idesc = umma_idesc_bf16(128, mode == 1 ? 64 : 128, 0, 1);
         for (int kk = 0; kk < 8; ++kk) {
           uint64_t bd = sdesc_sw128(smem_u32(b_s) + kk * 2048, 16384, 1024);
           umma_ts(tmem, tmem + 128 + kk * 8, bd, idesc, kk != 0);
@@ -87,7 +91,7 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_con
   bool ok = mbar_wait(&bar_mma, 0, ab);
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
-  const int ncol = mode == 0 ? 128 : 64;
+  const int ncol = mode == 1 ? 64 : 128;
   const int row = warp * 32 + lane;
   if (ok) {
     for (int c = 0; c < ncol / 32; ++c) {

@@ -223,7 +223,9 @@ int gemma_attn_last_launch_count(void);
  *           d [128][128] f32 = a * b^T.
  *   mode 1: p [128][128] bf16 staged through tensor memory, b [128][64] bf16 read
  *           MN-major; d [128][64] f32 = p * b.
- * a must be NULL-or-ignored in mode 1 and p in mode 0.
+ *   mode 2: as mode 1 with b [128][128] (two 64-column MN-major chunks, N = 128);
+ *           d [128][128] f32 = p * b.
+ * a must be NULL-or-ignored in modes 1 and 2, and p in mode 0.
  */
 int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const void* p, float* d,
                              void* stream);

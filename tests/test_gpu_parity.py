@@ -58,6 +58,19 @@ def test_umma_selftest_ts_mnmajor():
     np.testing.assert_allclose(d.cpu().numpy(), ref, rtol=1e-4, atol=1e-3)
 
 
+def test_umma_selftest_ts_mnmajor_two_chunks():
+    # N = 128: the second 64-column chunk is reached through the descriptor's leading
+    # byte offset, as in the paired kernel's N = 256 value product.
+    rng = np.random.default_rng(3)
+    p = W.f32_to_bf16_bits(rng.standard_normal((128, 128), dtype=np.float32))
+    v = W.f32_to_bf16_bits(rng.standard_normal((128, 128), dtype=np.float32))
+    d = torch.zeros((128, 128), dtype=torch.float32, device="cuda")
+    G.gemma_attn_selftest_umma(2, None, dev_bf16(v), dev_bf16(p), d)
+    torch.cuda.synchronize()
+    ref = _bf16_to_f64(p) @ _bf16_to_f64(v)
+    np.testing.assert_allclose(d.cpu().numpy(), ref, rtol=1e-4, atol=1e-3)
+
+
 # ------------------------------------------------------------------ prefill
 
 def _check_prefill(layer, seq_lens, seed=0, pos_start=0, rows=None):
