@@ -73,6 +73,7 @@ struct PrefillCfg {
   static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
   static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages * kStageBytes >= 4 * 32 * (64 * 4 + 16), "epilogue staging fits in the ring");
   static_assert(!PAIR || D >= 128, "paired form needs at least two 64-dim chunks");
   static_assert(kKStages >= 1 && kVStages >= 1 && kStages >= 2, "ring shape");
   static_assert(kPvN <= 256, "PV MMA width");
@@ -474,28 +475,55 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
       const bool valid = grow < len;
       const int tok = tok0 + grow;
-      const size_t obase = ((size_t)tok * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv;
+      // Each warp stages its 32 rows, 64 columns at a time, in its own slice of the ring
+      // (idle once o_ready has fired: every load was consumed by a finished MMA) and then
+      // writes whole 16-byte segments of few rows per store, instead of one scattered
+      // segment per row.
+      {
+        constexpr int kCols = 64;
+        const int esz = args.out_f32 ? 4 : 2;
+        const int row_bytes = kCols * esz;  // 128 or 256
+        const int stride = row_bytes + 16;  // padded: conflict-free 16-byte row writes
+        uint8_t* stg = ring + quad * 32 * (kCols * 4 + 16);
+        const int lanes_per_row = row_bytes / 16;
+        const int rows_per_pass = 32 / lanes_per_row;
+        const int seg = lane % lanes_per_row;
+        const int ncols = args.head_dim - vpart * Cfg::kDv;  // below kDv only for head_dim 32
 #pragma unroll 1
-      for (int c = 0; c < Cfg::kDv / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
-        tmem_ld_wait();
-        if (valid && vpart * Cfg::kDv + c * 32 < args.head_dim) {
+        for (int c = 0; c < Cfg::kDv / kCols; ++c) {
+          uint32_t o[kCols];
+          tmem_ld_x32(tmem + lane_off + kColO + c * kCols, o);
+          tmem_ld_x32(tmem + lane_off + kColO + c * kCols + 32, o + 32);
+          tmem_ld_wait();
+          uint8_t* mine = stg + lane * stride;
           if (args.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out) + obase + c * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                   __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+            for (int i = 0; i < kCols / 4; ++i)
+              *reinterpret_cast<float4*>(mine + 16 * i) =
+                  make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                              __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
           } else {
-            uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.out) + obase + c * 32);
+            for (int i = 0; i < kCols / 8; ++i) {
+              uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+              for (int k = 0; k < 4; ++k)
+                w[k] = pack_bf16x2(__uint_as_float(o[8 * i + 2 * k]) * inv_l, __uint_as_float(o[8 * i + 2 * k + 1]) * inv_l);
+              *reinterpret_cast<uint4*>(mine + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
+          __syncwarp();
+          const int col = c * kCols + seg * (16 / esz);
+          for (int r = lane / lanes_per_row; r < 32; r += rows_per_pass) {
+            const int trow = row0 + quad * 32 + r;  // in-sequence row
+            if (trow < len && col < ncols) {
+              const size_t off =
+                  ((size_t)(tok0 + trow) * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv + col;
+              *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(args.out) + off * esz) =
+                  *reinterpret_cast<const uint4*>(stg + r * stride + seg * 16);
+            }
+          }
+          __syncwarp();
         }
       }
       if (valid && vpart == 0 && args.lse != nullptr)
