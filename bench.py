@@ -74,27 +74,78 @@ def measured_peaks():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons sampled during the timed region.
+
+    Polls NVML (the library nvidia-smi reads) from a thread every ~2 ms, so that even a
+    region of a few tens of milliseconds gets samples; falls back to `nvidia-smi -lms`
+    when NVML is unavailable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.rows = []
+        self.thread = None
+        self.stop = False
+        self.source = None
+
+    def _nvml_start(self):
+        import threading
+        import pynvml as nv
+        import torch
+        nv.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+        h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        max_sm = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+        def sample():
+            sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.rows.append((sm, max_sm, ["Active" if r & b else "Not Active" for b in bits]))
+
+        def loop():
+            while not self.stop:
+                try:
+                    sample()
+                except Exception:
+                    return
+                time.sleep(0.002)
+
+        sample()
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
 
     def __enter__(self):
+        try:
+            self._nvml_start()
+            return self
+        except Exception:
+            self.rows = []
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                  "-i", str(self.idx)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi"
+            t0 = time.time()  # let the first sample land before the timed region starts
+            while time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -103,27 +154,28 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        rows = []
-        try:
-            for line in open(self.path):
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-                except ValueError:
-                    continue
-        finally:
+        rows = list(self.rows)
+        if self.path is not None:
             try:
-                os.unlink(self.path)
-            except Exception:
-                pass
+                for line in open(self.path):
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                    except ValueError:
+                        continue
+            finally:
+                try:
+                    os.unlink(self.path)
+                except Exception:
+                    pass
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower().startswith("active")})
+        reasons = sorted({self.NAMES[i] for _, _, flags in rows for i, f in enumerate(flags)
+                          if f.lower().startswith("active")})
         return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": self.source}
 
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
@@ -247,27 +299,21 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
     import global_interleaved_layers_b200 as G
+
+    from global_interleaved_layers_b200.replicas import Replicas
 
     world, rank, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    reps = Replicas(backend="nccl", timeout_s=120)  # process group only when WORLD_SIZE > 1
     dev = torch.device("cuda", local)
     peaks = measured_peaks()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        reps.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reps.max_over_ranks(x, dev)
 
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -436,8 +482,7 @@ def main():
         result["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(result), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    reps.close()
 
 
 def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
