@@ -467,8 +467,8 @@ def main():
         },
         "roofline": {"bound": "tensor", "achieved": g_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": g_tflops / peak_t, "traffic": ncu_traffic(), "traffic_unit": "bytes per launch",
-                     "kernel": "prefill_kernel<512> (global layer; timed call also launches the two small "
-                               "rotated-side-copy kernels)",
+                     "kernel": "prefill_kernel<512> (global layer; timed call also launches the small "
+                               "rotated-side-copy kernel)",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},

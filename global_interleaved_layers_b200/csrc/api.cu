@@ -177,14 +177,14 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
     RopeArgs ra;
     ra.positions = positions; ra.tokens = total_tokens; ra.d = d; ra.r = L.r; ra.chunk_mask = L.mask;
     ra.n_out = L.n_out; ra.log2_base = log2_base;
+    // queries and keys in one launch (the angles of a token serve both)
     ra.src = static_cast<const uint16_t*>(q); ra.dst = qside; ra.heads = Hq;
-    if (launch_rope_side(ra, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
-    ++t_launches;
-    ra.src = static_cast<const uint16_t*>(k); ra.dst = kside; ra.heads = Hkv;
+    ra.src2 = static_cast<const uint16_t*>(k); ra.dst2 = kside; ra.heads2 = Hkv;
     if (launch_rope_side(ra, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
     ++t_launches;
     if (pad) {
-      ra.src = static_cast<const uint16_t*>(global ? k : v); ra.dst = vpad; ra.r = 0;
+      ra.heads2 = 0; ra.src2 = nullptr; ra.dst2 = nullptr;
+      ra.src = static_cast<const uint16_t*>(global ? k : v); ra.dst = vpad; ra.heads = Hkv; ra.r = 0;
       if (launch_rope_side(ra, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
       ++t_launches;
     }

@@ -38,6 +38,9 @@ cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cud
 struct RopeArgs {
   const uint16_t* src;      // [T, H, d] bf16
   uint16_t* dst;            // [T, H, n_out] bf16, n_out = popcount(chunk_mask) * 64
+  const uint16_t* src2;     // optional second tensor [T, H2, d] (the keys), same rotation
+  uint16_t* dst2;           // [T, H2, n_out]
+  int heads2;               // 0: no second tensor
   const int32_t* positions; // [T]
   int tokens;
   int heads;

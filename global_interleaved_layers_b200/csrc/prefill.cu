@@ -16,7 +16,10 @@
 //              running max only raised when it grows by more than 2^8, P written back to
 //              TMEM as bf16 over the scores, epilogue O / l.
 // The MMA order is S(j), PV(j-1), S(j+1), PV(j), ... so the tensor core works on
-// S(j+1) while the softmax warps turn S(j) into P(j).
+// S(j+1) while the softmax warps turn S(j) into P(j). The kernel is persistent: each
+// CTA (pair) stays resident and walks a list of work units, so barrier setup, TMEM
+// allocation and teardown happen once, and the next unit's Q load and first score tiles
+// overlap the current unit's last value product and epilogue.
 //
 // Paired form (PAIR): the two query heads of a GQA pair share every K and V tile. Two
 // CTAs on two SMs form a cluster; the even CTA issues 256-row MMAs (tcgen05 cta_group::2)
@@ -73,7 +76,6 @@ struct PrefillCfg {
   static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
   static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kStages * kStageBytes >= 4 * 32 * (64 * 4 + 16), "epilogue staging fits in the ring");
   static_assert(!PAIR || D >= 128, "paired form needs at least two 64-dim chunks");
   static_assert(kKStages >= 1 && kVStages >= 1 && kStages >= 2, "ring shape");
   static_assert(kPvN <= 256, "PV MMA width");
@@ -83,8 +85,10 @@ struct __align__(8) Barriers {
   uint64_t q_full;
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t pv_done;
-  uint64_t o_ready;  // one phase: every PV of the work unit has finished
+  uint64_t pv_done[2];  // by tile parity: PV(t) completes phase t >> 1 of pv_done[t & 1]
+  uint64_t q_empty;  // per unit: its last score MMA finished, Q may be replaced
+  uint64_t o_ready;  // per unit: its last value MMA finished
+  uint64_t o_empty;  // per unit: the softmax warps have read O out
   uint64_t mma_done;
   uint64_t ring_full[kMaxStages];
   uint64_t ring_empty[kMaxStages];
@@ -109,6 +113,22 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 
 }  // namespace
 
+// Persistent form: the grid holds as many CTAs (or CTA pairs) as can be resident, and
+// each walks a fixed list of work units. Unit u (0 .. U-1, heaviest query tiles first)
+// goes to cluster u mod C in forward order on even rounds and reverse order on odd
+// rounds (C = number of clusters), which balances the causal tile counts. Every role
+// of a CTA walks the same list; barrier phases continue across units:
+//   ring stages          continuous (st, ph) in the producer and the MMA issuer
+//   s_full / p_full /    tile counter g over all tiles this CTA has processed; each is
+//   pv_done              a pair of barriers indexed by tile parity, so that a waiter's
+//                        phase is never two behind (after a unit's last PV the next
+//                        unit's first S waits for the PV before it)
+//   q_full / q_empty /   one phase per unit: Q landed / the unit's last score MMA
+//   o_ready / o_empty    finished (Q may be replaced) / the unit's last value MMA
+//                        finished / the softmax warps have read O out (the next
+//                        unit's first value MMA may overwrite it)
+// The next unit's Q load and its first two score tiles overlap the current unit's
+// last value product and epilogue.
 template <int D, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap qs_map,
@@ -124,40 +144,58 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- which work unit ----
-  // blockIdx.x = (head_unit * kSplit + vpart) [* 2 + rank in the pair]
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
-  const int unit_x = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int vpart = unit_x % Cfg::kSplit;
-  const int head = PAIR ? (unit_x / Cfg::kSplit) * 2 + (int)rank : unit_x / Cfg::kSplit;
-  const int slot = blockIdx.y;
-  const int seq = slot % args.num_seqs;
-  const int qt = args.max_qtiles - 1 - slot / args.num_seqs;  // heaviest tiles first
-  const int tok0 = args.cu_seqlens[seq];
-  const int len = args.cu_seqlens[seq + 1] - tok0;
-  if (qt == 0 && vpart == 0 && head == 0 && threadIdx.x == 0 && (len > args.max_seqlen || len < 1))
-    atomicOr(&g_status, kStatusSeqlen);
-  // Both CTAs of a pair share (seq, qt), so they leave here together, before any
-  // cluster-wide synchronisation.
-  if (qt * kBM >= len) return;
-  const int row0 = qt * kBM;
-  const int kvh = head / args.group;
   const int is_local = args.is_local;
-  int kt_lo, kt_hi;
-  kv_tile_range(is_local, args.window, len, qt, kBM, kBN, &kt_lo, &kt_hi);
-  const int ntiles = kt_hi - kt_lo;
+
+  // ---- the unit schedule ----
+  const int units_x = (PAIR ? args.num_q_heads / 2 : args.num_q_heads) * Cfg::kSplit;
+  const int num_units = units_x * args.num_seqs * args.max_qtiles;
+  const int nclusters = (int)gridDim.x / (PAIR ? 2 : 1);
+  const int cid = (int)blockIdx.x / (PAIR ? 2 : 1);
+  struct Unit {
+    int head, vpart, qt, tok0, len, row0, kvh, kt_lo, ntiles;
+  };
+  // Unit of round r for this cluster; false when the round has none or the unit is empty
+  // (a query tile past its sequence's end).
+  auto unit_of_round = [&](int r, Unit& w) -> bool {
+    const int u = r * nclusters + ((r & 1) ? nclusters - 1 - cid : cid);
+    if (u >= num_units) return false;
+    const int slot = u / units_x, ux = u % units_x;
+    const int seq = slot % args.num_seqs;
+    w.qt = args.max_qtiles - 1 - slot / args.num_seqs;
+    w.vpart = ux % Cfg::kSplit;
+    w.head = PAIR ? (ux / Cfg::kSplit) * 2 + (int)rank : ux / Cfg::kSplit;
+    w.tok0 = args.cu_seqlens[seq];
+    w.len = args.cu_seqlens[seq + 1] - w.tok0;
+    if (w.qt * kBM >= w.len) return false;
+    w.row0 = w.qt * kBM;
+    w.kvh = w.head / args.group;
+    int hi;
+    kv_tile_range(is_local, args.window, w.len, w.qt, kBM, kBN, &w.kt_lo, &hi);
+    w.ntiles = hi - w.kt_lo;
+    return true;
+  };
+  const int nrounds = (num_units + nclusters - 1) / nclusters;
 
   if (threadIdx.x == 0) {
+    // sequence-length check, once per sequence, by the CTA that owns round 0 of cluster 0
+    if (cid == 0 && leader)
+      for (int sq = 0; sq < args.num_seqs; ++sq) {
+        const int n = args.cu_seqlens[sq + 1] - args.cu_seqlens[sq];
+        if (n > args.max_seqlen || n < 1) atomicOr(&g_status, kStatusSeqlen);
+      }
     const uint32_t load_arrivals = PAIR ? 2u : 1u;  // pair: both producers register their bytes
     mbar_init(&bars->q_full, load_arrivals);
+    mbar_init(&bars->q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_full[b], PAIR ? 8 : 4);  // one arrival per softmax warp (of both CTAs)
     }
-    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->pv_done[0], 1);
+    mbar_init(&bars->pv_done[1], 1);
     mbar_init(&bars->o_ready, 1);
+    mbar_init(&bars->o_empty, PAIR ? 8 : 4);
     mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&bars->ring_full[s], load_arrivals);
@@ -203,63 +241,78 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       };
       auto rot_idx = [&](int c) { return __popc(args.rot_mask & ((1u << c) - 1)); };
 
-      expect(&bars->q_full, Cfg::kQBytes);
-      for (int c = 0; c < Cfg::kQChunks; ++c) {
-        if ((args.rot_mask >> c) & 1) load(q_smem + c * kChunkBytes, &qs_map, &bars->q_full, rot_idx(c) * kChunk, head, tok0 + row0);
-        else load(q_smem + c * kChunkBytes, &q_map, &bars->q_full, c * kChunk, head, tok0 + row0);
-      }
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
       bool ok = true;
-      for (int jj = 0; jj <= ntiles && ok; ++jj) {
-        if (jj < ntiles) {  // K stages of tile jj
-          const int key0 = tok0 + (kt_lo + jj) * kBN;
-          for (int s = 0; s < Cfg::kKStages && ok; ++s) {
-            ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
-            if (!ok) break;
-            expect(&bars->ring_full[st], Cfg::kStageBytes);
-            uint8_t* dst = ring + st * Cfg::kStageBytes;
-            if constexpr (PAIR) {
-              // chunks kKPerStage * s + sub of this CTA's 64 keys
-              for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
-                const int c = Cfg::kKPerStage * s + sub;
-                if ((args.rot_mask >> c) & 1)
-                  load(dst + sub * Cfg::kKChunkBytes, &ks64_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh,
-                       key0 + 64 * (int)rank);
-                else
-                  load(dst + sub * Cfg::kKChunkBytes, &k64_map, &bars->ring_full[st], c * kChunk, kvh,
-                       key0 + 64 * (int)rank);
+      int unit_iter = 0, q_issued = 0;
+      for (int r = 0; r < nrounds && ok; ++r) {
+        Unit w;
+        if (!unit_of_round(r, w)) continue;
+        // Q of this unit replaces the previous unit's once its last score MMA finished
+        if (unit_iter > 0) {
+          ok = mbar_wait(&bars->q_empty, (uint32_t)(unit_iter - 1) & 1u, abort_flag);
+          if (!ok) break;
+        }
+        expect(&bars->q_full, Cfg::kQBytes);
+        for (int c = 0; c < Cfg::kQChunks; ++c) {
+          if ((args.rot_mask >> c) & 1)
+            load(q_smem + c * kChunkBytes, &qs_map, &bars->q_full, rot_idx(c) * kChunk, w.head, w.tok0 + w.row0);
+          else
+            load(q_smem + c * kChunkBytes, &q_map, &bars->q_full, c * kChunk, w.head, w.tok0 + w.row0);
+        }
+        ++q_issued;
+        for (int jj = 0; jj <= w.ntiles && ok; ++jj) {
+          if (jj < w.ntiles) {  // K stages of tile jj
+            const int key0 = w.tok0 + (w.kt_lo + jj) * kBN;
+            for (int s = 0; s < Cfg::kKStages && ok; ++s) {
+              ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
+              if (!ok) break;
+              expect(&bars->ring_full[st], Cfg::kStageBytes);
+              uint8_t* dst = ring + st * Cfg::kStageBytes;
+              if constexpr (PAIR) {
+                // chunks kKPerStage * s + sub of this CTA's 64 keys
+                for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
+                  const int c = Cfg::kKPerStage * s + sub;
+                  if ((args.rot_mask >> c) & 1)
+                    load(dst + sub * Cfg::kKChunkBytes, &ks64_map, &bars->ring_full[st], rot_idx(c) * kChunk, w.kvh,
+                         key0 + 64 * (int)rank);
+                  else
+                    load(dst + sub * Cfg::kKChunkBytes, &k64_map, &bars->ring_full[st], c * kChunk, w.kvh,
+                         key0 + 64 * (int)rank);
+                }
+              } else {
+                const int c = s;
+                if ((args.rot_mask >> c) & 1) load(dst, &ks_map, &bars->ring_full[st], rot_idx(c) * kChunk, w.kvh, key0);
+                else load(dst, &k_map, &bars->ring_full[st], c * kChunk, w.kvh, key0);
               }
-            } else {
-              const int c = s;
-              if ((args.rot_mask >> c) & 1) load(dst, &ks_map, &bars->ring_full[st], rot_idx(c) * kChunk, kvh, key0);
-              else load(dst, &k_map, &bars->ring_full[st], c * kChunk, kvh, key0);
+              next();
             }
-            next();
+          }
+          if (jj >= 1) {  // V stages of tile jj-1 (this unit's output columns)
+            const int key0 = w.tok0 + (w.kt_lo + jj - 1) * kBN;
+            for (int s = 0; s < Cfg::kVStages && ok; ++s) {
+              ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
+              if (!ok) break;
+              expect(&bars->ring_full[st], Cfg::kStageBytes);
+              // this CTA's column chunks of V stage s: the pair's two CTAs hold adjacent groups
+              for (int sub = 0; sub < Cfg::kVPerStage; ++sub) {
+                const int c = ((PAIR ? 2 * s + (int)rank : s) * Cfg::kVPerStage) + sub;
+                load(ring + st * Cfg::kStageBytes + sub * kChunkBytes, &v_map, &bars->ring_full[st],
+                     w.vpart * Cfg::kDv + c * kChunk, w.kvh, key0);
+              }
+              next();
+            }
           }
         }
-        if (jj >= 1) {  // V stages of tile jj-1 (this unit's output columns)
-          const int key0 = tok0 + (kt_lo + jj - 1) * kBN;
-          for (int s = 0; s < Cfg::kVStages && ok; ++s) {
-            ok = mbar_wait(&bars->ring_empty[st], ph ^ 1u, abort_flag);
-            if (!ok) break;
-            expect(&bars->ring_full[st], Cfg::kStageBytes);
-            // this CTA's column chunks of V stage s: the pair's two CTAs hold adjacent groups
-            for (int sub = 0; sub < Cfg::kVPerStage; ++sub) {
-              const int c = ((PAIR ? 2 * s + (int)rank : s) * Cfg::kVPerStage) + sub;
-              load(ring + st * Cfg::kStageBytes + sub * kChunkBytes, &v_map, &bars->ring_full[st],
-                   vpart * Cfg::kDv + c * kChunk, kvh, key0);
-            }
-            next();
-          }
-        }
+        ++unit_iter;
       }
       // Let the copies counted on this CTA's barriers land before the CTA can exit: the
-      // last kStages loads are the only ones that may still be in flight. (st, ph) is the
-      // next slot to fill; each slot's most recent fill completed the phase of parity
-      // ph ^ 1 (the wrap inside next() flips ph for the slots filled this round). In the
-      // paired form the odd CTA's copies complete on the even CTA's barriers, whose MMA
-      // consumes every one of them before the final cluster barrier.
+      // last kStages ring loads and the last Q load are the only ones that may still be
+      // in flight. (st, ph) is the next slot to fill; each slot's most recent fill
+      // completed the phase of parity ph ^ 1 (the wrap inside next() flips ph for the
+      // slots filled this round). In the paired form the odd CTA's copies complete on the
+      // even CTA's barriers, whose MMA consumes every one of them before the final
+      // cluster barrier.
       if (!PAIR || leader) {
         for (int s = 0; s < Cfg::kStages; ++s) {
           if (!mbar_try_wait(&bars->ring_full[st], ph ^ 1u)) {
@@ -268,6 +321,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           }
           next();
           (void)s;
+        }
+        if (q_issued > 0 && !mbar_try_wait(&bars->q_full, (uint32_t)(q_issued - 1) & 1u)) {
+          unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&bars->q_full, (uint32_t)(q_issued - 1) & 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {}
         }
       }
     }
@@ -284,71 +341,86 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(ring), 16, 1024);
       // V is MN-major: 64-column chunks of a stage are kChunkBytes apart (leading offset)
       const uint64_t v_desc0 = sdesc_sw128(smem_u32(ring), kChunkBytes, 1024);
+      auto commit_both = [&](uint64_t* bar) {
+        if constexpr (PAIR) umma_commit_pair_both(bar);
+        else umma_commit(bar);
+      };
       int st = 0; uint32_t ph = 0;
       auto next = [&]() { if (++st == Cfg::kStages) { st = 0; ph ^= 1u; } };
-      bool ok = wait_bar<PAIR>(&bars->q_full, 0, abort_flag);
-      for (int jj = 0; jj <= ntiles && ok; ++jj) {
-        if (jj < ntiles) {
-          const int b = jj & 1;
-          const uint32_t s_col = b ? kColS1 : kColS0;
-          if (jj >= 2) ok = wait_bar<PAIR>(&bars->pv_done, (uint32_t)(jj - 2) & 1u, abort_flag);
-          tc_fence_after();
-          for (int s = 0; s < Cfg::kKStages && ok; ++s) {
-            ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
-            if (!ok) break;
+      bool ok = true;
+      int g = 0;  // tiles of earlier units
+      int unit_iter = 0;
+      for (int r = 0; r < nrounds && ok; ++r) {
+        Unit w;
+        if (!unit_of_round(r, w)) continue;
+        ok = wait_bar<PAIR>(&bars->q_full, (uint32_t)unit_iter & 1u, abort_flag);
+        for (int jj = 0; jj <= w.ntiles && ok; ++jj) {
+          if (jj < w.ntiles) {
+            const int t = g + jj;
+            const int b = t & 1;
+            const uint32_t s_col = b ? kColS1 : kColS0;
+            // S(t) overwrites the buffer whose P fed PV(t-2)
+            if (t >= 2) ok = wait_bar<PAIR>(&bars->pv_done[t & 1], (uint32_t)((t - 2) >> 1) & 1u, abort_flag);
             tc_fence_after();
-            const uint64_t kd = k_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
+            for (int s = 0; s < Cfg::kKStages && ok; ++s) {
+              ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              const uint64_t kd = k_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
 #pragma unroll
-            for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
-              const int c = Cfg::kKPerStage * s + sub;
-              const uint64_t qd = q_desc0 + (uint64_t)((c * kChunkBytes) >> 4);
-              const uint64_t kds = kd + (uint64_t)((sub * Cfg::kKChunkBytes) >> 4);
+              for (int sub = 0; sub < Cfg::kKPerStage; ++sub) {
+                const int c = Cfg::kKPerStage * s + sub;
+                const uint64_t qd = q_desc0 + (uint64_t)((c * kChunkBytes) >> 4);
+                const uint64_t kds = kd + (uint64_t)((sub * Cfg::kKChunkBytes) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < kChunk / 16; ++kk) {
-                if constexpr (PAIR) umma_ss_pair(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
-                else umma_ss(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
+                for (int kk = 0; kk < kChunk / 16; ++kk) {
+                  if constexpr (PAIR) umma_ss_pair(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
+                  else umma_ss(tmem + s_col, qd + 2 * kk, kds + 2 * kk, idesc_qk, (c | kk) != 0);
+                }
               }
+              commit_both(&bars->ring_empty[st]);
+              next();
             }
-            if constexpr (PAIR) umma_commit_pair_both(&bars->ring_empty[st]);
-            else umma_commit(&bars->ring_empty[st]);
-            next();
-          }
-          if (!ok) break;
-          if constexpr (PAIR) umma_commit_pair_both(&bars->s_full[b]);
-          else umma_commit(&bars->s_full[b]);
-        }
-        if (jj >= 1) {
-          const int pj = jj - 1;
-          const int pb = pj & 1;
-          const uint32_t p_col = pb ? kColS1 : kColS0;
-          ok = wait_bar<PAIR>(&bars->p_full[pb], (uint32_t)(pj >> 1) & 1u, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          for (int s = 0; s < Cfg::kVStages && ok; ++s) {
-            ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
             if (!ok) break;
-            tc_fence_after();
-            const uint64_t vd = v_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
-            const uint32_t o_col = kColO + s * PV_N;
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              if constexpr (PAIR) umma_ts_pair(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, (pj | kk) != 0);
-              else umma_ts(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, (pj | kk) != 0);
-            }
-            if constexpr (PAIR) umma_commit_pair_both(&bars->ring_empty[st]);
-            else umma_commit(&bars->ring_empty[st]);
-            next();
+            commit_both(&bars->s_full[b]);
+            if (jj == w.ntiles - 1) commit_both(&bars->q_empty);  // the unit's last read of Q
           }
-          if (!ok) break;
-          if constexpr (PAIR) umma_commit_pair_both(&bars->pv_done);
-          else umma_commit(&bars->pv_done);
+          if (jj >= 1) {
+            const int pt = g + jj - 1;
+            const int pb = pt & 1;
+            const uint32_t p_col = pb ? kColS1 : kColS0;
+            ok = wait_bar<PAIR>(&bars->p_full[pb], (uint32_t)(pt >> 1) & 1u, abort_flag);
+            if (!ok) break;
+            // the unit's first value MMA overwrites O: the previous unit's epilogue has read it
+            if (jj == 1 && unit_iter > 0) {
+              ok = wait_bar<PAIR>(&bars->o_empty, (uint32_t)(unit_iter - 1) & 1u, abort_flag);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            for (int s = 0; s < Cfg::kVStages && ok; ++s) {
+              ok = wait_bar<PAIR>(&bars->ring_full[st], ph, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              const uint64_t vd = v_desc0 + (uint64_t)((st * Cfg::kStageBytes) >> 4);
+              const uint32_t o_col = kColO + s * PV_N;
+#pragma unroll
+              for (int kk = 0; kk < kBN / 16; ++kk) {
+                const bool acc = (jj - 1) != 0 || kk != 0;
+                if constexpr (PAIR) umma_ts_pair(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, acc);
+                else umma_ts(tmem + o_col, tmem + p_col + kk * 8, vd + 128 * kk, idesc_pv, acc);
+              }
+              commit_both(&bars->ring_empty[st]);
+              next();
+            }
+            if (!ok) break;
+            commit_both(&bars->pv_done[pt & 1]);
+          }
         }
-      }
-      // The epilogue waits on o_ready, a single-phase barrier: softmax warps skip pv_done
-      // phases, so a parity wait on pv_done could not tell the last phase from an older one.
-      if (ok) {
-        if constexpr (PAIR) umma_commit_pair_both(&bars->o_ready);
-        else umma_commit(&bars->o_ready);
+        if (!ok) break;
+        // O of the unit is final once every value MMA issued so far has finished
+        commit_both(&bars->o_ready);
+        g += w.ntiles;
+        ++unit_iter;
       }
       // All MMAs issued by this thread are complete once mma_done fires.
       if constexpr (PAIR) umma_commit_pair_local(&bars->mma_done);
@@ -362,172 +434,165 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float scale_log2 = args.softmax_scale * 1.4426950408889634f;
-    float m_used = -INFINITY;
-    float l_sum = 0.f;
-    const int grow = row0 + row;  // in-sequence offset of this thread's query row
     bool ok = true;
-    for (int jj = 0; jj < ntiles && ok; ++jj) {
-      const int b = jj & 1;
-      const uint32_t s_col = b ? kColS1 : kColS0;
-      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->s_full[b], (uint32_t)(jj >> 1) & 1u, abort_flag));
+    int g = 0;
+    int unit_iter = 0;
+    for (int r = 0; r < nrounds && ok; ++r) {
+      Unit w;
+      if (!unit_of_round(r, w)) continue;
+      float m_used = -INFINITY;
+      float l_sum = 0.f;
+      const int grow = w.row0 + row;  // in-sequence offset of this thread's query row
+      for (int jj = 0; jj < w.ntiles && ok; ++jj) {
+        const int t = g + jj;
+        const int b = t & 1;
+        const uint32_t s_col = b ? kColS1 : kColS0;
+        ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->s_full[b], (uint32_t)(t >> 1) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kBN];
+        uint32_t* tr = reinterpret_cast<uint32_t*>(sv);
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
+        tmem_ld_wait();
+        const int kt = w.kt_lo + jj;
+        // A key tile that runs past the end of the sequence holds the next sequence's
+        // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
+        const bool partial = (kt + 1) * kBN > w.len ||
+                             kv_tile_class(is_local, args.window, w.len, w.qt, kt, kBM, kBN) != kTileFull;
+        // Masked tiles are scaled here (masked entries -inf); full tiles keep raw scores and
+        // fold the scale into the exponent's FFMA (scale > 0, so the max commutes with it).
+        // Eight partial maxima keep the reduction off one long dependency chain.
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+        if (partial) {
+          const int k0 = kt * kBN;
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const int key = k0 + c;
+            const bool vis = key <= grow && (!is_local || key > grow - args.window);
+            sv[c] = vis ? sv[c] * scale_log2 : -INFINITY;
+            mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+        }
+        const float coef = partial ? 1.f : scale_log2;
+        float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        if (!partial) m_tile *= scale_log2;
+        // Raise the running max only when it grows by more than 2^8 (or was empty); P
+        // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
+        float alpha = 1.f;
+        bool rescale_o = false;
+        if (m_tile > m_used + kRescaleThreshold || (m_used == -INFINITY && m_tile > -INFINITY)) {
+          if (m_used != -INFINITY) {
+            alpha = fast_exp2(m_used - m_tile);
+            l_sum *= alpha;
+            rescale_o = true;
+          }
+          m_used = m_tile;
+        }
+        // P(t) goes over S(t) right away: that buffer's previous P (tile t-2) was consumed
+        // by PV(t-2), which finished before S(t) was computed.
+        const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+        uint32_t p[kBN / 2];
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kBN / 2; ++c) {
+          const float p0 = fast_exp2(fmaf(sv[2 * c], coef, -m_sub));
+          const float p1 = fast_exp2(fmaf(sv[2 * c + 1], coef, -m_sub));
+          rs4[c & 3] += p0 + p1;
+          p[c] = pack_bf16x2(p0, p1);
+        }
+        l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        tmem_st_x32(tmem + lane_off + s_col, p);
+        tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
+        // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
+        // lane needs it, each lane with its own factor (1 for lanes that do not). O may only
+        // be touched once PV(t-1) has finished; without a rescale the warp does not wait,
+        // since PV(t) is issued after PV(t-1) and the tensor core runs them in order. The
+        // parity wait is exact: PV(t-3) finished before S(t-1) was issued, and PV(t+1) needs
+        // this warp's p_full(t+1) arrival, so PV(t-1) is the only phase of its barrier that
+        // can still be pending. A unit's first tile never rescales (m_used starts empty).
+        const bool rescale_warp = __any_sync(0xffffffffu, rescale_o);
+        if (rescale_warp && jj >= 1) {
+          ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag));
+          if (!ok) {
+            tmem_st_wait();  // the P stores land before the teardown frees TMEM
+            break;
+          }
+          tc_fence_after();
+        }
+        if (rescale_warp) {
+#pragma unroll 1
+          for (int c = 0; c < Cfg::kDv / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();  // every lane's P and O stores precede the warp's single arrival
+        if (lane == 0) {
+          if (!PAIR || leader) mbar_arrive(&bars->p_full[b]);
+          else mbar_arrive_cluster(smem_u32(&bars->p_full[b]) & kPeerBitMask);
+        }
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->o_ready, (uint32_t)unit_iter & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float t[kBN];
-      uint32_t* tr = reinterpret_cast<uint32_t*>(t);
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
-      tmem_ld_wait();
-      const int kt = kt_lo + jj;
-      // A key tile that runs past the end of the sequence holds the next sequence's
-      // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
-      const bool partial = (kt + 1) * kBN > len ||
-                           kv_tile_class(is_local, args.window, len, qt, kt, kBM, kBN) != kTileFull;
-      // Masked tiles are scaled here (masked entries -inf); full tiles keep raw scores and
-      // fold the scale into the exponent's FFMA (scale > 0, so the max commutes with it).
-      // Eight partial maxima keep the reduction off one long dependency chain.
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-      if (partial) {
-        const int k0 = kt * kBN;
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const int key = k0 + c;
-          const bool vis = key <= grow && (!is_local || key > grow - args.window);
-          t[c] = vis ? t[c] * scale_log2 : -INFINITY;
-          mx8[c & 7] = fmaxf(mx8[c & 7], t[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], t[c]);
-      }
-      const float coef = partial ? 1.f : scale_log2;
-      float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      if (!partial) m_tile *= scale_log2;
-      // Raise the running max only when it grows by more than 2^8 (or was empty); P
-      // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
-      float alpha = 1.f;
-      bool rescale_o = false;
-      if (m_tile > m_used + kRescaleThreshold || (m_used == -INFINITY && m_tile > -INFINITY)) {
-        if (m_used != -INFINITY) {
-          alpha = fast_exp2(m_used - m_tile);
-          l_sum *= alpha;
-          rescale_o = true;
-        }
-        m_used = m_tile;
-      }
-      // P(jj) goes over S(jj) right away: that buffer's previous P (tile jj-2) was consumed
-      // by PV(jj-2), which finished before S(jj) was computed. Only the O rescale has to
-      // wait for PV(jj-1), so the exponentials stay off the PV -> softmax -> PV chain.
-      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t p[kBN / 2];
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < kBN / 2; ++c) {
-        const float p0 = fast_exp2(fmaf(t[2 * c], coef, -m_sub));
-        const float p1 = fast_exp2(fmaf(t[2 * c + 1], coef, -m_sub));
-        rs4[c & 3] += p0 + p1;
-        p[c] = pack_bf16x2(p0, p1);
-      }
-      l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      tmem_st_x32(tmem + lane_off + s_col, p);
-      tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
-      // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
-      // lane needs it, each lane with its own factor (1 for lanes that do not). O may only
-      // be touched once PV(jj-1) has finished; without a rescale the warp does not wait,
-      // since PV(jj) is issued after PV(jj-1) and the tensor core runs them in order.
-      // The parity wait is exact: S(jj) was issued after PV(jj-2) finished, and PV(jj)
-      // needs this warp's p_full(jj) arrival below, so PV(jj-1) is the only pv_done phase
-      // that can still be pending.
-      const bool rescale_warp = __any_sync(0xffffffffu, rescale_o);
-      if (rescale_warp && jj >= 1) {
-        ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done, (uint32_t)(jj - 1) & 1u, abort_flag));
-        if (!ok) {
-          tmem_st_wait();  // the P stores land before the teardown frees TMEM
-          break;
-        }
-        tc_fence_after();
-      }
-      if (rescale_warp) {
-#pragma unroll 1
-        for (int c = 0; c < Cfg::kDv / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();  // every lane's P and O stores precede the warp's single arrival
-      if (lane == 0) {
-        if (!PAIR || leader) mbar_arrive(&bars->p_full[b]);
-        else mbar_arrive_cluster(smem_u32(&bars->p_full[b]) & kPeerBitMask);
-      }
-    }
-    if (ok && ntiles > 0)
-      ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->o_ready, 0u, abort_flag));
-    if (ok) {
-      tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      const bool valid = grow < len;
-      const int tok = tok0 + grow;
-      // Each warp stages its 32 rows, 64 columns at a time, in its own slice of the ring
-      // (idle once o_ready has fired: every load was consumed by a finished MMA) and then
-      // writes whole 16-byte segments of few rows per store, instead of one scattered
-      // segment per row.
-      {
-        constexpr int kCols = 64;
-        const int esz = args.out_f32 ? 4 : 2;
-        const int row_bytes = kCols * esz;  // 128 or 256
-        const int stride = row_bytes + 16;  // padded: conflict-free 16-byte row writes
-        uint8_t* stg = ring + quad * 32 * (kCols * 4 + 16);
-        const int lanes_per_row = row_bytes / 16;
-        const int rows_per_pass = 32 / lanes_per_row;
-        const int seg = lane % lanes_per_row;
-        const int ncols = args.head_dim - vpart * Cfg::kDv;  // below kDv only for head_dim 32
+      const bool valid = grow < w.len;
+      const int tok = w.tok0 + grow;
+      const size_t obase = ((size_t)tok * args.num_q_heads + w.head) * args.head_dim + w.vpart * Cfg::kDv;
 #pragma unroll 1
-        for (int c = 0; c < Cfg::kDv / kCols; ++c) {
-          uint32_t o[kCols];
-          tmem_ld_x32(tmem + lane_off + kColO + c * kCols, o);
-          tmem_ld_x32(tmem + lane_off + kColO + c * kCols + 32, o + 32);
-          tmem_ld_wait();
-          uint8_t* mine = stg + lane * stride;
-          if (args.out_f32) {
+      for (int c = 0; c < Cfg::kDv / 64; ++c) {
+        uint32_t o[64];
+        tmem_ld_x32(tmem + lane_off + kColO + c * 64, o);
+        tmem_ld_x32(tmem + lane_off + kColO + c * 64 + 32, o + 32);
+        tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < kCols / 4; ++i)
-              *reinterpret_cast<float4*>(mine + 16 * i) =
-                  make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                              __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
-          } else {
+        for (int h = 0; h < 2; ++h) {
+          const int col = c * 64 + h * 32;
+          const uint32_t* oh = o + h * 32;
+          if (valid && w.vpart * Cfg::kDv + col < args.head_dim) {
+            if (args.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out) + obase + col);
 #pragma unroll
-            for (int i = 0; i < kCols / 8; ++i) {
-              uint32_t w[4];
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(oh[4 * i]) * inv_l, __uint_as_float(oh[4 * i + 1]) * inv_l,
+                                     __uint_as_float(oh[4 * i + 2]) * inv_l, __uint_as_float(oh[4 * i + 3]) * inv_l);
+            } else {
+              uint32_t wd[16];
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                w[k] = pack_bf16x2(__uint_as_float(o[8 * i + 2 * k]) * inv_l, __uint_as_float(o[8 * i + 2 * k + 1]) * inv_l);
-              *reinterpret_cast<uint4*>(mine + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int i = 0; i < 16; ++i)
+                wd[i] = pack_bf16x2(__uint_as_float(oh[2 * i]) * inv_l, __uint_as_float(oh[2 * i + 1]) * inv_l);
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.out) + obase + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
             }
           }
-          __syncwarp();
-          const int col = c * kCols + seg * (16 / esz);
-          for (int r = lane / lanes_per_row; r < 32; r += rows_per_pass) {
-            const int trow = row0 + quad * 32 + r;  // in-sequence row
-            if (trow < len && col < ncols) {
-              const size_t off =
-                  ((size_t)(tok0 + trow) * args.num_q_heads + head) * args.head_dim + vpart * Cfg::kDv + col;
-              *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(args.out) + off * esz) =
-                  *reinterpret_cast<const uint4*>(stg + r * stride + seg * 16);
-            }
-          }
-          __syncwarp();
         }
       }
-      if (valid && vpart == 0 && args.lse != nullptr)
-        args.lse[(size_t)head * args.total_tokens + tok] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
+      if (valid && w.vpart == 0 && args.lse != nullptr)
+        args.lse[(size_t)w.head * args.total_tokens + tok] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
+      // O has been read out: the next unit's first value MMA may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (!PAIR || leader) mbar_arrive(&bars->o_empty);
+        else mbar_arrive_cluster(smem_u32(&bars->o_empty) & kPeerBitMask);
+      }
+      g += w.ntiles;
+      ++unit_iter;
     }
   }
 
@@ -549,17 +614,45 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
 }
 
 template <int D, bool PAIR>
+constexpr int Cfg_smem() { return PrefillCfg<D, PAIR>::kSmemBytes; }
+
+// Clusters (pairs) or CTAs of prefill_kernel<D, PAIR> that fit on the device at once,
+// computed once per device.
+template <int D, bool PAIR>
+static int resident_clusters(const cudaLaunchConfig_t& cfg) {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t c = cfg;
+    c.gridDim = dim3(2, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_kernel<D, PAIR>, &c) != cudaSuccess) n = 0;
+  } else {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel<D, PAIR>, kThreads,
+                                                      Cfg_smem<D, PAIR>()) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      n = per_sm * sms;
+  }
+  cached[dev] = n;
+  return n;
+}
+
+template <int D, bool PAIR>
 cudaError_t launch_prefill_t(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
   using Cfg = PrefillCfg<D, PAIR>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(args.num_q_heads * Cfg::kSplit, args.num_seqs * args.max_qtiles);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = stream;
@@ -572,6 +665,14 @@ cudaError_t launch_prefill_t(const PrefillMaps& maps, const PrefillArgs& args, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
+  // Persistent grid: as many CTAs (pairs) as can be resident at once, at most one per unit.
+  const long long units = (long long)(PAIR ? args.num_q_heads / 2 : args.num_q_heads) * Cfg::kSplit *
+                          args.num_seqs * args.max_qtiles;
+  if (units == 0) return cudaSuccess;
+  const int resident = resident_clusters<D, PAIR>(cfg);
+  if (resident < 1) return cudaErrorInvalidConfiguration;
+  const long long clusters = units < resident ? units : resident;
+  cfg.gridDim = dim3((unsigned)(clusters * (PAIR ? 2 : 1)), 1, 1);
   return cudaLaunchKernelEx(&cfg, prefill_kernel<D, PAIR>, maps.q, maps.qs, maps.k, maps.ks, maps.v, maps.k64,
                             maps.ks64, args);
 }

@@ -38,9 +38,45 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 
 }  // namespace
 
+// Rotates (or copies) the 8 pairs j0..j0+7 of every head of one token of one tensor,
+// four heads at a time so that eight 16-byte loads are in flight before any store.
+__device__ __forceinline__ void rope_heads(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
+                                           int heads, int tok, int d, int n_out, int j0, int col0, int col1,
+                                           bool pad, const float* c, const float* s) {
+  const int half = d / 2;
+  for (int h0 = 0; h0 < heads; h0 += 4) {
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (h0 + k < heads) {
+        const uint16_t* p = src + ((size_t)tok * heads + h0 + k) * d;
+        a[k] = __ldg(reinterpret_cast<const uint4*>(p + j0));
+        b[k] = __ldg(reinterpret_cast<const uint4*>(p + j0 + half));
+      }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (h0 + k < heads) {
+        uint16_t* q = dst + ((size_t)tok * heads + h0 + k) * n_out;
+        float x0[8], x1[8], y0[8], y1[8];
+        unpack8(a[k], x0);
+        unpack8(b[k], x1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          y0[e] = x0[e] * c[e] - x1[e] * s[e];
+          y1[e] = x0[e] * s[e] + x1[e] * c[e];
+        }
+        if (col0 >= 0) *reinterpret_cast<uint4*>(q + col0) = pack8(y0);
+        if (col1 >= 0) *reinterpret_cast<uint4*>(q + col1) = pack8(y1);
+        if (pad)
+          for (int z = d; z < 64; z += 8) *reinterpret_cast<uint4*>(q + z) = make_uint4(0, 0, 0, 0);
+      }
+  }
+}
+
 // One thread per (token, group of 8 consecutive pairs j0..j0+7): it computes the 8
-// angles once and rotates those pairs in every head of the token with 16-byte loads
-// and stores of both halves (dims j0.. and j0 + d/2 ..).
+// angles once and rotates those pairs in every head of the token, for the queries and
+// (in the same launch) the keys, with 16-byte loads and stores of both halves (dims
+// j0.. and j0 + d/2 ..).
 __global__ void rope_side_kernel(RopeArgs a) {
   const int half = a.d / 2;
   const int groups = half / 8;
@@ -58,22 +94,8 @@ __global__ void rope_side_kernel(RopeArgs a) {
     if (j0 + e < a.r) rope_cos_sin((double)a.positions[tok], rope_inv_freq_turns(j0 + e, a.d, a.log2_base), &c[e], &s[e]);
   }
   const bool pad = a.d < 64 && j0 == 0;  // this thread also zeroes the padding columns d .. 63
-  for (int h = 0; h < a.heads; ++h) {
-    const uint16_t* src = a.src + ((size_t)tok * a.heads + h) * a.d;
-    uint16_t* dst = a.dst + ((size_t)tok * a.heads + h) * a.n_out;
-    float x0[8], x1[8], y0[8], y1[8];
-    unpack8(*reinterpret_cast<const uint4*>(src + j0), x0);
-    unpack8(*reinterpret_cast<const uint4*>(src + j0 + half), x1);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      y0[e] = x0[e] * c[e] - x1[e] * s[e];
-      y1[e] = x0[e] * s[e] + x1[e] * c[e];
-    }
-    if (col0 >= 0) *reinterpret_cast<uint4*>(dst + col0) = pack8(y0);
-    if (col1 >= 0) *reinterpret_cast<uint4*>(dst + col1) = pack8(y1);
-    if (pad)
-      for (int z = a.d; z < 64; z += 8) *reinterpret_cast<uint4*>(dst + z) = make_uint4(0, 0, 0, 0);
-  }
+  rope_heads(a.src, a.dst, a.heads, tok, a.d, a.n_out, j0, col0, col1, pad, c, s);
+  if (a.heads2 > 0) rope_heads(a.src2, a.dst2, a.heads2, tok, a.d, a.n_out, j0, col0, col1, pad, c, s);
 }
 
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream) {
