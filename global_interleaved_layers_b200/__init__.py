@@ -69,9 +69,10 @@ _lib.gemma_attn_tile_plan.argtypes = [_I, _I, _P, _I, _I, _I, _P, ctypes.c_int64
 _lib.gemma_attn_decode_noalloc.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_check.argtypes = [_P]
 _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
+_lib.gemma_attn_selftest_timeout.argtypes = [_P, _P]
 for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_attn_decode",
            "gemma_attn_decode_num_splits", "gemma_attn_combine", "gemma_attn_tile_plan", "gemma_attn_check",
-           "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc"):
+           "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc", "gemma_attn_selftest_timeout"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -190,6 +191,10 @@ def gemma_attn_check(stream=None) -> None:
 def gemma_attn_selftest_umma(mode: int, a, b, p, d, stream=None) -> None:
     _check(_lib.gemma_attn_selftest_umma(mode, _ptr(a), _ptr(b), _ptr(p), _ptr(d), _stream(stream)),
            "gemma_attn_selftest_umma")
+
+
+def gemma_attn_selftest_timeout(gave_up, stream=None) -> None:
+    _check(_lib.gemma_attn_selftest_timeout(_ptr(gave_up), _stream(stream)), "gemma_attn_selftest_timeout")
 
 
 def raw_call(name: str, *args) -> int:

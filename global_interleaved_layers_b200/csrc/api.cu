@@ -360,6 +360,14 @@ int gemma_attn_check(void* stream_) {
   return GEMMA_ATTN_OK;
 }
 
+int gemma_attn_selftest_timeout(int32_t* gave_up, void* stream_) {
+  t_launches = 0;
+  if (!gave_up) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (launch_timeout_selftest(gave_up, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
+  t_launches = 1;
+  return GEMMA_ATTN_OK;
+}
+
 int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const void* p, float* d, void* stream_) {
   t_launches = 0;
   if (mode < 0 || mode > 2 || !b || !d || (mode == 0 && !a) || (mode != 0 && !p))

@@ -80,5 +80,6 @@ struct CombineArgs {
   int out_f32;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+cudaError_t launch_timeout_selftest(int* gave_up, cudaStream_t stream);
 
 }  // namespace gattn

@@ -120,3 +120,30 @@ cudaError_t launch_umma_selftest(const CUtensorMap& a, const CUtensorMap& b, con
 }
 
 }  // namespace gattn
+
+namespace gattn {
+
+// One CTA waits on an mbarrier that nothing arrives at. The bounded wait gives up after
+// its limit, records a timeout in the device status word and the kernel returns: the
+// path every pipeline wait takes when a peer role never signals.
+__global__ void timeout_selftest_kernel(int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, &abort_flag);
+    *gave_up = ok ? 0 : 1;
+  }
+}
+
+cudaError_t launch_timeout_selftest(int* gave_up, cudaStream_t stream) {
+  timeout_selftest_kernel<<<1, 32, 0, stream>>>(gave_up);
+  return cudaGetLastError();
+}
+
+}  // namespace gattn

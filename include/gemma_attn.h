@@ -230,6 +230,15 @@ int gemma_attn_last_launch_count(void);
 int gemma_attn_selftest_umma(int32_t mode, const void* a, const void* b, const void* p, float* d,
                              void* stream);
 
+/*
+ * Diagnostic of the failure path: launches one CTA that waits on an mbarrier nothing
+ * arrives at. Every wait in the kernels is bounded (about 2 s of the GPU's global timer);
+ * this one runs out, records a timeout in the device status word (the next
+ * gemma_attn_check returns GEMMA_ATTN_ERR_TIMEOUT and clears it) and writes 1 to the
+ * device int *gave_up. The context stays usable. The pages have no counterpart to it.
+ */
+int gemma_attn_selftest_timeout(int32_t* gave_up, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

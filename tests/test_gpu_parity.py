@@ -58,6 +58,20 @@ def test_umma_selftest_ts_mnmajor():
     np.testing.assert_allclose(d.cpu().numpy(), ref, rtol=1e-4, atol=1e-3)
 
 
+def test_bounded_wait_times_out_and_context_survives():
+    # A wait on a barrier nothing arrives at gives up after its limit, the status word
+    # reports the timeout once, and later launches run normally.
+    G.gemma_attn_check()
+    flag = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    G.gemma_attn_selftest_timeout(flag)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_check()
+    assert e.value.status == G.ERR_TIMEOUT
+    assert int(flag.item()) == 1
+    G.gemma_attn_check()  # cleared
+    test_umma_selftest_ss_kmajor()
+
+
 def test_umma_selftest_ts_mnmajor_two_chunks():
     # N = 128: the second 64-column chunk is reached through the descriptor's leading
     # byte offset, as in the paired kernel's N = 256 value product.
