@@ -544,40 +544,51 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
 
         log(f"decode kind={layer.kind}")
 
-        def one():
-            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
-            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+        def measure(layout):
+            def one():
+                G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+                G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
 
-        for _ in range(args.warmup):
-            one()
-        torch.cuda.synchronize()
-        G.gemma_attn_check()
-        evs = []
-        dec_evs = []
-        barrier()
-        for _ in range(args.steps):
-            flush_l2()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e2 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
-            e1.record(stream)
-            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
-            e2.record(stream)
-            evs.append((e0, e2))
-            dec_evs.append((e0, e1))
-        torch.cuda.synchronize()
-        barrier()
-        ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
-        dec_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dec_evs])))
-        nbytes = W.decode_cache_bytes(B, wl.cache_lens, layer)
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        name = "global_decode" if layer.kind == W.GLOBAL else "local_decode"
-        res[name] = {"gbs": gbs, "ms": ms, "decode_kernel_ms": dec_ms, "bytes": nbytes, "splits": splits,
-                     "frac_of_hbm": gbs / peaks["hbm_gbs"],
-                     "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} ctx={ctx} " + ("K=V contiguous" if layer.k_eq_v
-                                                                             else f"ring W={layer.window}")}
+            for _ in range(args.warmup):
+                one()
+            torch.cuda.synchronize()
+            G.gemma_attn_check()
+            evs = []
+            dec_evs = []
+            barrier()
+            for _ in range(args.steps):
+                flush_l2()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e2 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+                e1.record(stream)
+                G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+                e2.record(stream)
+                evs.append((e0, e2))
+                dec_evs.append((e0, e1))
+            torch.cuda.synchronize()
+            G.gemma_attn_check()
+            barrier()
+            ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+            dec_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dec_evs])))
+            nbytes = W.decode_cache_bytes(B, wl.cache_lens, layer)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            rotated = bool(layout & G.CACHE_KEYS_ROTATED)
+            return {"gbs": gbs, "ms": ms, "decode_kernel_ms": dec_ms, "bytes": nbytes, "splits": splits,
+                    "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                    "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} ctx={ctx} " + (
+                        "K=V contiguous" if layer.k_eq_v else
+                        f"ring W={layer.window}, cached keys {'stored rotated' if rotated else 'un-rotated'}")}
+
+        if layer.kind == W.GLOBAL:
+            res["global_decode"] = measure(layout)
+        else:
+            # the serving layout keeps local keys rotated in the cache; the un-rotated cache
+            # (the kernel rotates every key) is reported beside it
+            res["local_decode"] = measure(layout | G.CACHE_KEYS_ROTATED)
+            res["local_decode_unrotated_cache"] = measure(layout)
         del kc, vc
         torch.cuda.empty_cache()
     return res

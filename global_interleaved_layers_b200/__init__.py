@@ -25,6 +25,7 @@ LOCAL = 0
 GLOBAL = 1
 CACHE_CONTIGUOUS = 0
 CACHE_RING = 1
+CACHE_KEYS_ROTATED = 0x100  # OR-ed into the layout (local layers): cached keys stored rotated
 OUT_BF16 = 0
 OUT_F32 = 1
 

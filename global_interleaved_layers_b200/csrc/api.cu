@@ -274,6 +274,9 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   if (!q || !new_k || !k_cache || !cache_seqlens || !partial_o || !partial_lse) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (batch < 1 || n_q < 1 || num_splits < 1 || max_cache_len < 0) return GEMMA_ATTN_ERR_INVALID_ARG;
+  const bool keys_rotated = (cache_layout & GEMMA_ATTN_CACHE_KEYS_ROTATED) != 0;
+  if (keys_rotated && global) return GEMMA_ATTN_ERR_INVALID_ARG;  // the K=V tensor is also the values
+  cache_layout &= ~GEMMA_ATTN_CACHE_KEYS_ROTATED;
   if (cache_layout != GEMMA_ATTN_CACHE_CONTIGUOUS && cache_layout != GEMMA_ATTN_CACHE_RING)
     return GEMMA_ATTN_ERR_INVALID_ARG;
   if (cache_layout == GEMMA_ATTN_CACHE_RING && (global || cache_capacity != params->window))
@@ -296,6 +299,7 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   a.batch = batch; a.n_q = n_q; a.num_q_heads = params->num_q_heads; a.num_kv_heads = params->num_kv_heads;
   a.head_dim = params->head_dim; a.is_local = global ? 0 : 1; a.window = global ? 0 : params->window;
   a.ring = cache_layout == GEMMA_ATTN_CACHE_RING; a.capacity = cache_capacity; a.num_splits = num_splits;
+  a.keys_rotated = keys_rotated ? 1 : 0;
   a.r = rotated_pairs(params->rope_p, params->head_dim);
   a.log2_base = log2((double)params->rope_base);
   a.softmax_scale = params->softmax_scale;

@@ -264,8 +264,8 @@ decode_tc_kernel(DecodeArgs a) {
       __syncthreads();
     }
 
-    // ---- rotated copy for scores
-    if (r > 0) {
+    // ---- rotated copy for scores (with pre-rotated cached keys only the new tokens' rows)
+    if (r > 0 && (!a.keys_rotated || pos0 + kCK > len)) {
       if (kv_same) {
         // non-rotated dims that share a 16-dim k-step with rotated ones are copied first
         if (r % 16 != 0) {
@@ -299,7 +299,7 @@ decode_tc_kernel(DecodeArgs a) {
           if (kv_same) {
             rbuf[u * RST + sj * 16 + (j % 16)] = y0;
             rbuf[u * RST + sp * 16 + ((j + HALF) % 16)] = y1;
-          } else {
+          } else if (!a.keys_rotated || pos0 + u >= len) {
             kd[u * KST + j] = y0;
             kd[u * KST + j + HALF] = y1;
           }
@@ -524,8 +524,9 @@ static cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
 namespace {
 
 constexpr int kWB = 16;        // keys per warp block
-// header: mbarriers [warps][stages] at 0, abort flag at 128, merge maxima [warps][8]
-// at 256 and sums [warps][8] after them
+// header: mbarriers [warps][stages] at 0, abort flag at 128, value-stage mbarriers
+// [warps][value stages] at 160 (split form), merge maxima [warps][8] at 256 and sums
+// [warps][8] after them
 constexpr int kWMgM = 256;
 __host__ __device__ constexpr int wmg_l(int nw) { return kWMgM + nw * 32; }
 __host__ __device__ constexpr int wheader(int nw) { return (wmg_l(nw) + nw * 32 + 127) / 128 * 128; }
@@ -538,9 +539,10 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 
 __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
-// Shared-memory carve-up of decode_warp_kernel<D, NS, NW>; r is the rotated pair count and nrk
-// the number of rotated 16-dim k-steps kept in the per-warp rotated copy (K=V layers).
-template <int D, int NS, int NW>
+// Shared-memory carve-up of decode_warp_kernel<D, NS, NW, NSV>; r is the rotated pair count
+// and nrk the number of rotated 16-dim k-steps kept in the per-warp rotated copy (K=V
+// layers). NS key stages per warp; separate-V layers add NSV value stages.
+template <int D, int NS, int NW, int NSV>
 struct DecWLayout {
   static constexpr int KST = D + 8;  // bf16 row stride of key / value / query rows
   static constexpr int RED = D + 4;  // fp32 row stride of the merge buffer
@@ -558,7 +560,7 @@ struct DecWLayout {
     regions = itf + align128((size_t)rr2 * 8);
     k_off = 0;
     v_off = (size_t)NS * kWB * KST * 2;
-    rot_off = kv_same ? v_off : 2 * v_off;
+    rot_off = kv_same ? v_off : v_off + (size_t)NSV * kWB * KST * 2;
     ast_off = rot_off + (kv_same ? (size_t)kWB * rst * 2 : 0);
     const int nwords = kv_same ? 8 * ((r + 15) / 16) : (r + 1) / 2;
     region = align128(ast_off + (size_t)(nwords > 0 ? nwords : 1) * 16);
@@ -573,12 +575,16 @@ __host__ __device__ inline bool rotated_kstep(int s, int half, int r) {
 
 }  // namespace
 
-template <int D, int NS, int NW>
+template <int D, int NS, int NW, int NSV>
 __global__ void __launch_bounds__(NW * 32)
 decode_warp_kernel(DecodeArgs a) {
-  using L = DecWLayout<D, NS, NW>;
+  using L = DecWLayout<D, NS, NW, NSV>;
   constexpr int kWWarps = NW;
   constexpr int kWStages = NS;  // ring stages per warp
+  // Split form (separate-V layers only): key rows and value rows stream through their
+  // own stages with their own barriers, so the next block's keys are in flight while
+  // this block's values are used and the next values while the next keys are rotated.
+  constexpr bool kSplit = NSV < NS;
   constexpr int HALF = D / 2;
   constexpr int KST = L::KST;
   constexpr int NKS = D / 16;
@@ -606,7 +612,7 @@ decode_warp_kernel(DecodeArgs a) {
   const int RST = lay.rst;
 
   extern __shared__ __align__(128) uint8_t dsm[];
-  static_assert(kWWarps * NS * 8 <= 128, "mbarriers overflow their header slot");
+  static_assert(kWWarps * NS * 8 <= 128 && (!kSplit || kWWarps * NSV * 8 <= 96), "mbarriers overflow their header slots");
   uint64_t* bars = reinterpret_cast<uint64_t*>(dsm);  // [warps][stages]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + 128);
   float* mg_m = reinterpret_cast<float*>(dsm + kWMgM);  // [warps][8]
@@ -621,6 +627,7 @@ decode_warp_kernel(DecodeArgs a) {
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(region + lay.rot_off);
   float4* ast = reinterpret_cast<float4*>(region + lay.ast_off);  // this warp's block anchors
   uint64_t* wbar = bars + warp * kWStages;
+  uint64_t* vbar = reinterpret_cast<uint64_t*>(dsm + 160) + warp * NSV;  // split form
 
   // blocks of this warp: warp, warp + NW, ... of the split's ceil((v_hi - v_lo) / 16)
   const int nblk = (v_hi - v_lo + kWB - 1) / kWB;
@@ -650,15 +657,44 @@ decode_warp_kernel(DecodeArgs a) {
       bulk_load(dst, src, D * 2, &wbar[st]);
     }
   };
+  // Split form: the key rows (kv = 0) or value rows (kv = 1) of block `itx`, lanes 0..15.
+  auto issue_half = [&](int itx, int kv) {
+    const int st = kv ? itx % NSV : itx % kWStages;
+    uint64_t* bar = kv ? &vbar[st] : &wbar[st];
+    const int v0 = v_lo + (warp + kWWarps * itx) * kWB;
+    const int nvalid = min(kWB, v_hi - v0);
+    fence_proxy_async_smem();
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nvalid * D * 2));
+    __syncwarp();
+    const int row = lane;
+    if (row < nvalid) {
+      const int pos = first + v0 + row;
+      const uint16_t* src;
+      if (pos < len) {
+        const size_t slot = a.ring ? (size_t)(pos % a.capacity) : (size_t)pos;
+        src = (kv ? a.v_cache : a.k_cache) + (((size_t)b * a.num_kv_heads + kvh) * a.capacity + slot) * D;
+      } else {
+        src = (kv ? a.new_v : a.new_k) + (((size_t)b * a.n_q + (pos - len)) * a.num_kv_heads + kvh) * D;
+      }
+      bulk_load((kv ? vst : kst) + (st * kWB + row) * KST, src, D * 2, bar);
+    }
+  };
 
   if (lane == 0) {
     for (int s = 0; s < kWStages; ++s) mbar_init(&wbar[s], 1);
+    if constexpr (kSplit)
+      for (int s = 0; s < NSV; ++s) mbar_init(&vbar[s], 1);
     fence_barrier_init();
   }
   if (tid == 0) *abort_flag = 0;
   __syncwarp();
   // the first blocks stream in while the CTA prepares queries and angle tables
-  for (int s = 0; s < kWStages && s < my_n; ++s) issue(s);
+  if constexpr (kSplit) {
+    for (int s = 0; s < kWStages && s < my_n; ++s) issue_half(s, 0);
+    for (int s = 0; s < NSV && s < my_n; ++s) issue_half(s, 1);
+  } else {
+    for (int s = 0; s < kWStages && s < my_n; ++s) issue(s);
+  }
 
   // rotated queries (bf16); rows R..7 are zero
   for (int idx = tid; idx < 8 * HALF; idx += kWWarps * 32) {
@@ -731,11 +767,11 @@ decode_warp_kernel(DecodeArgs a) {
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     uint16_t* kd = kst + st * kWB * KST;
-    uint16_t* vdw = kv_same ? kd : vst + st * kWB * KST;
+    uint16_t* vdw = kv_same ? kd : vst + (kSplit ? it % NSV : st) * kWB * KST;
     const int v0 = v_lo + (warp + kWWarps * it) * kWB;
     const int nvalid = min(kWB, v_hi - v0);
     const int pos0 = first + v0;
-    if (nvalid < kWB) {  // value rows past the split end: zero, so that P = 0 meets finite values
+    if (!kSplit && nvalid < kWB) {  // value rows past the split end: zero, so that P = 0 meets finite values
       for (int idx = lane; idx < (kWB - nvalid) * (D / 8); idx += 32) {
         const int row = nvalid + idx / (D / 8), c8 = idx % (D / 8);
         *reinterpret_cast<uint4*>(vdw + row * KST + c8 * 8) = make_uint4(0, 0, 0, 0);
@@ -746,11 +782,13 @@ decode_warp_kernel(DecodeArgs a) {
     // keys from the angle of the block's first key, stepping by theta_j per key. That
     // anchor angle is exact every 16th block and otherwise the previous block's anchor
     // advanced by 16 NW theta_j (the warp's stride); all loads come first.
-    if (r > 0) {
+    // With pre-rotated cached keys only a block holding new tokens is rotated (those rows
+    // only), from an exact anchor since the recurrence skipped the blocks before it.
+    if (r > 0 && (!a.keys_rotated || pos0 + kWB > len)) {
       uint16_t* dst0 = kv_same ? rbuf : kd;
       const int dst_hi = kv_same ? 16 * c16 : HALF;
       const int dst_st = kv_same ? RST : KST;
-      const bool exact = (it & 15) == 0;
+      const bool exact = (it & 15) == 0 || a.keys_rotated;
       for (int w = lane; w < nwords; w += 32) {
         const int j = 2 * w;
         uint32_t w0[kWB], w1[kWB];
@@ -779,8 +817,10 @@ decode_warp_kernel(DecodeArgs a) {
           const float x10 = __uint_as_float(w1[u] << 16), x11 = __uint_as_float(w1[u] & 0xFFFF0000u);
           const uint32_t o0 = pack_bf16x2(x00 * ac[0] - x10 * as[0], x01 * ac[1] - x11 * as[1]);
           const uint32_t o1 = pack_bf16x2(x00 * as[0] + x10 * ac[0], x01 * as[1] + x11 * ac[1]);
-          *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + j) = o0;
-          *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + dst_hi + j) = o1;
+          if (!a.keys_rotated || pos0 + u >= len) {
+            *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + j) = o0;
+            *reinterpret_cast<uint32_t*>(dst0 + u * dst_st + dst_hi + j) = o1;
+          }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const float nc = ac[e] * sc[e] - as[e] * ss[e];
@@ -814,6 +854,11 @@ decode_warp_kernel(DecodeArgs a) {
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[e] += (sch[0][e] + sch[1][e]) + sch[2][e];
+    }
+
+    if constexpr (kSplit) {
+      __syncwarp();  // every lane is done with this block's key rows
+      if (it + kWStages < my_n) issue_half(it + kWStages, 0);
     }
 
     // ---- 3. mask and online softmax; fragment element e: key g + 8 * (e >> 1), row 2t + (e & 1)
@@ -861,6 +906,19 @@ decode_warp_kernel(DecodeArgs a) {
     const uint32_t pb0 = movmatrix_trans(p01);
     const uint32_t pb1 = movmatrix_trans(p23);
 
+    if constexpr (kSplit) {
+      ok = mbar_wait(&vbar[it % NSV], (uint32_t)(it / NSV) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (nvalid < kWB) {  // value rows past the split end: zero, so that P = 0 meets finite values
+        for (int idx = lane; idx < (kWB - nvalid) * (D / 8); idx += 32) {
+          const int row = nvalid + idx / (D / 8), c8 = idx % (D / 8);
+          *reinterpret_cast<uint4*>(vdw + row * KST + c8 * 8) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+    }
+
     // ---- 4. O^T += V^T P^T over the whole head dim
     {
       const uint32_t vbase = smem_u32(vdw) + vfrag;
@@ -872,15 +930,27 @@ decode_warp_kernel(DecodeArgs a) {
       }
     }
     __syncwarp();  // every lane is done with this stage and the rotated copy
-    if (it + kWStages < my_n) issue(it + kWStages);
+    if constexpr (kSplit) {
+      if (it + NSV < my_n) issue_half(it + NSV, 1);
+    } else {
+      if (it + kWStages < my_n) issue(it + kWStages);
+    }
   }
   // Copies still in flight after an early exit land before the warp moves on.
   if (!ok && lane == 0) {
-    for (int k = it; k < my_n && k < it + kWStages; ++k) {
+    // key (or combined) stages issued for blocks it .. it + NS - 1; in the split form the
+    // keys may already be one block further (issued after this block's scores)
+    for (int k = it; k < my_n && k < it + kWStages + (kSplit ? 1 : 0); ++k) {
       const uint32_t par = (uint32_t)(k / kWStages) & 1u;
       const unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(&wbar[k % kWStages], par) && globaltimer_ns() - t0 < kWaitLimitNs) {}
     }
+    if constexpr (kSplit)
+      for (int k = it; k < my_n && k < it + NSV; ++k) {
+        const uint32_t par = (uint32_t)(k / NSV) & 1u;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&vbar[k % NSV], par) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+      }
   }
 
   // ---- merge the warps' (max, sum, O) and write this split's partial
@@ -937,25 +1007,25 @@ decode_warp_kernel(DecodeArgs a) {
   }
 }
 
-template <int D, int NS, int NW>
+template <int D, int NS, int NW, int NSV>
 static size_t decode_warp_smem(const DecodeArgs& a) {
   const bool kv_same = a.v_cache == nullptr;
   int nrk = 0;
   if (kv_same)
     for (int s = 0; s < D / 16; ++s)
       if (rotated_kstep(s, D / 2, a.r)) ++nrk;
-  return DecWLayout<D, NS, NW>(kv_same, a.r, nrk).total;
+  return DecWLayout<D, NS, NW, NSV>(kv_same, a.r, nrk).total;
 }
 
-template <int D, int NS, int NW>
+template <int D, int NS, int NW, int NSV>
 static cudaError_t launch_decode_warp(const DecodeArgs& a, cudaStream_t stream) {
-  const size_t smem = decode_warp_smem<D, NS, NW>(a);
+  const size_t smem = decode_warp_smem<D, NS, NW, NSV>(a);
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<D, NS, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<D, NS, NW, NSV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.num_splits, a.num_kv_heads, a.batch);
-  decode_warp_kernel<D, NS, NW><<<grid, NW * 32, smem, stream>>>(a);
+  decode_warp_kernel<D, NS, NW, NSV><<<grid, NW * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -963,10 +1033,11 @@ static cudaError_t launch_decode_warp(const DecodeArgs& a, cudaStream_t stream) 
 int decode_max_rows(int head_dim) { return head_dim >= 512 ? 32 : 64; }
 
 // Decode kernel variant for a shape: the warp-independent kernel for up to 8 rows (the
-// first of 8 warps x 2 ring stages, 8 x 1, 4 x 1 that fits), the
+// first that fits of 8 warps x 2 ring stages, 8 warps x 2 key stages + 1 value stage
+// (separate-V layers), 8 x 1, 4 x 1), the
 // CTA-wide kernel with 16, 32 or 64 row slots above that; kDecNone when no variant fits
 // in shared memory.
-enum DecodeVariant { kDecNone = 0, kDecWarp8x2, kDecWarp8x1, kDecWarp4x1, kDecTc2, kDecTc4, kDecTc8 };
+enum DecodeVariant { kDecNone = 0, kDecWarp8x2, kDecWarp8x2s, kDecWarp8x1, kDecWarp4x1, kDecTc2, kDecTc4, kDecTc8 };
 
 template <int D>
 static int decode_variant_d(const DecodeArgs& a) {
@@ -977,9 +1048,10 @@ static int decode_variant_d(const DecodeArgs& a) {
     for (int s = 0; s < D / 16; ++s)
       if (rotated_kstep(s, D / 2, a.r)) ++nrk;
   if (R <= 8) {
-    if (decode_warp_smem<D, 2, 8>(a) <= kMaxSmem) return kDecWarp8x2;
-    if (decode_warp_smem<D, 1, 8>(a) <= kMaxSmem) return kDecWarp8x1;
-    if (decode_warp_smem<D, 1, 4>(a) <= kMaxSmem) return kDecWarp4x1;
+    if (decode_warp_smem<D, 2, 8, 2>(a) <= kMaxSmem) return kDecWarp8x2;
+    if (!kv_same && decode_warp_smem<D, 2, 8, 1>(a) <= kMaxSmem) return kDecWarp8x2s;
+    if (decode_warp_smem<D, 1, 8, 1>(a) <= kMaxSmem) return kDecWarp8x1;
+    if (decode_warp_smem<D, 1, 4, 1>(a) <= kMaxSmem) return kDecWarp4x1;
     return kDecNone;
   }
   if (R <= 16) return dec_smem_bytes<D, 2>(!kv_same, nrk) <= kMaxSmem ? kDecTc2 : kDecNone;
@@ -991,9 +1063,10 @@ static int decode_variant_d(const DecodeArgs& a) {
 template <int D>
 static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t stream) {
   switch (decode_variant_d<D>(a)) {
-    case kDecWarp8x2: return launch_decode_warp<D, 2, 8>(a, stream);
-    case kDecWarp8x1: return launch_decode_warp<D, 1, 8>(a, stream);
-    case kDecWarp4x1: return launch_decode_warp<D, 1, 4>(a, stream);
+    case kDecWarp8x2: return launch_decode_warp<D, 2, 8, 2>(a, stream);
+    case kDecWarp8x2s: return launch_decode_warp<D, 2, 8, 1>(a, stream);
+    case kDecWarp8x1: return launch_decode_warp<D, 1, 8, 1>(a, stream);
+    case kDecWarp4x1: return launch_decode_warp<D, 1, 4, 1>(a, stream);
     case kDecTc2: return launch_decode_tc<D, 2>(a, stream);
     case kDecTc4: return launch_decode_tc<D, 4>(a, stream);
     case kDecTc8:

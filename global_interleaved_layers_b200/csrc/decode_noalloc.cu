@@ -80,6 +80,9 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (batch < 1 || n_q < 1 || num_splits < 1 || max_cache_len < 0 || cache_capacity < 1)
     return GEMMA_ATTN_ERR_INVALID_ARG;
+  const bool keys_rotated = (cache_layout & GEMMA_ATTN_CACHE_KEYS_ROTATED) != 0;
+  if (keys_rotated && global) return GEMMA_ATTN_ERR_INVALID_ARG;  // the K=V tensor is also the values
+  cache_layout &= ~GEMMA_ATTN_CACHE_KEYS_ROTATED;
   if (cache_layout != GEMMA_ATTN_CACHE_CONTIGUOUS && cache_layout != GEMMA_ATTN_CACHE_RING)
     return GEMMA_ATTN_ERR_INVALID_ARG;
   if (cache_layout == GEMMA_ATTN_CACHE_RING && (global || cache_capacity != params->window))
@@ -115,6 +118,7 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   a.batch = batch; a.n_q = n_q; a.num_q_heads = params->num_q_heads; a.num_kv_heads = params->num_kv_heads;
   a.head_dim = d; a.is_local = global ? 0 : 1; a.window = global ? 0 : params->window;
   a.ring = cache_layout == GEMMA_ATTN_CACHE_RING; a.capacity = cache_capacity; a.num_splits = num_splits;
+  a.keys_rotated = keys_rotated ? 1 : 0;
   a.r = rotated_pairs(params->rope_p, d);
   a.log2_base = log2((double)params->rope_base);
   a.softmax_scale = params->softmax_scale;

@@ -63,6 +63,7 @@ struct DecodeArgs {
   float* partial_lse;       // [splits, rows]
   int batch, n_q, num_q_heads, num_kv_heads, head_dim;
   int is_local, window, ring, capacity, num_splits;
+  int keys_rotated;         // cached keys are stored rotated: only new tokens' keys are rotated here
   int r;
   double log2_base;
   float softmax_scale;

@@ -53,7 +53,13 @@ enum {
 
 enum {
   GEMMA_ATTN_CACHE_CONTIGUOUS = 0, /* [batch, kv_heads, capacity, head_dim]; token p at row p */
-  GEMMA_ATTN_CACHE_RING = 1        /* [batch, kv_heads, window, head_dim]; token p at slot p mod window */
+  GEMMA_ATTN_CACHE_RING = 1,       /* [batch, kv_heads, window, head_dim]; token p at slot p mod window */
+  /* Flag OR-ed into cache_layout, LOCAL layers only (separate value tensor): the cached
+   * keys are stored already rotated for their positions, as they were when written
+   * (token p's key rotated by p-RoPE at position p); the call then rotates only the new
+   * tokens' keys. Without it the cache holds un-rotated keys. A GLOBAL layer's single K=V
+   * tensor serves as the values too, so its cache stays un-rotated. */
+  GEMMA_ATTN_CACHE_KEYS_ROTATED = 0x100
 };
 
 enum {
@@ -132,7 +138,9 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
  *              GEMMA_ATTN_CACHE_RING (LOCAL only): [batch, num_kv_heads, window, head_dim],
  *              token p at slot p mod window, holding the last min(len, window) tokens;
  *              cache_capacity must equal window.
- *              Caches hold un-rotated keys (GLOBAL: the K=V tensor).
+ *              Caches hold un-rotated keys (GLOBAL: the K=V tensor), or for LOCAL with
+ *              GEMMA_ATTN_CACHE_KEYS_ROTATED in cache_layout, keys rotated for their
+ *              positions (new_k is always un-rotated).
  *   v_cache    same layout as k_cache for LOCAL; NULL for GLOBAL.
  *   cache_seqlens [batch] int32 device: tokens already cached (>= 0).
  *   max_cache_len  upper bound on cache_seqlens (sizes the launch).

@@ -95,6 +95,15 @@ def test_decode_argument_errors():
     with pytest.raises(G.GemmaAttnError) as e:
         G.gemma_attn_decode(pg, fake, fake, None, fake, None, G.CACHE_CONTIGUOUS, 64, fake, 1, 5, 10, fake, fake, 1, 0)
     assert e.value.status == G.ERR_UNSUPPORTED
+    # a global layer's K=V cache cannot hold rotated keys (they are also the values)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_decode(pg, fake, fake, None, fake, None, G.CACHE_CONTIGUOUS | G.CACHE_KEYS_ROTATED, 64, fake,
+                            1, 1, 10, fake, fake, 1, 0)
+    assert e.value.status == G.ERR_INVALID_ARG
+    # unknown layout bits
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_decode(p, fake, fake, fake, fake, fake, G.CACHE_RING | 0x40, 64, fake, 1, 1, 10, fake, fake, 1, 0)
+    assert e.value.status == G.ERR_INVALID_ARG
     # 16 rows of a separate-V d = 512 layer: no decode variant fits in shared memory
     pl = _p(num_q_heads=16, num_kv_heads=1, head_dim=512, window=64)
     with pytest.raises(G.GemmaAttnError) as e:

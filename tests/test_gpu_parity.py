@@ -154,7 +154,18 @@ def test_prefill_seqlen_violation_reported():
 
 # ------------------------------------------------------------------ decode / verify + combine
 
-def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11):
+def _rotated_history(k_hist_b, n, layer):
+    """Cached rows 0..n-1 of one sequence's key history rotated for their positions by the
+    oracle's p-RoPE and rounded to bf16 (the pre-rotated cache layout); new rows stay."""
+    out = k_hist_b.copy()
+    for p in range(n):
+        for h in range(k_hist_b.shape[1]):
+            x = W.bf16_bits_to_f32(k_hist_b[p, h]).astype(np.float64)
+            out[p, h] = W.f32_to_bf16_bits(oracle.rope(x, layer.rope_p, layer.rope_base, p).astype(np.float32))
+    return out
+
+
+def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11, keys_rotated=False):
     B = len(cache_lens)
     Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
     rng_seed = seed
@@ -166,16 +177,18 @@ def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11):
     ref, ref_lse = oracle.decode(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
                                  q, k_hist, None if layer.k_eq_v else v_hist, cache_lens)
     max_len = max(cache_lens)
+    # the oracle always gets the un-rotated history; the GPU cache may hold rotated keys
+    k_cache_src = [_rotated_history(k_hist[b], cache_lens[b], layer) for b in range(B)] if keys_rotated else k_hist
     if layout == G.CACHE_RING:
         cap = layer.window
-        kc = np.stack([ring_from_history(k_hist[b][:cache_lens[b]], cap) for b in range(B)])
+        kc = np.stack([ring_from_history(k_cache_src[b][:cache_lens[b]], cap) for b in range(B)])
         vc = None if layer.k_eq_v else np.stack([ring_from_history(v_hist[b][:cache_lens[b]], cap) for b in range(B)])
     else:
         cap = max(max_len, 1)
         kc = np.zeros((B, Hkv, cap, d), np.uint16)
         vc = None if layer.k_eq_v else np.zeros((B, Hkv, cap, d), np.uint16)
         for b, n in enumerate(cache_lens):
-            kc[b, :, :n] = k_hist[b][:n].transpose(1, 0, 2)
+            kc[b, :, :n] = k_cache_src[b][:n].transpose(1, 0, 2)
             if vc is not None:
                 vc[b, :, :n] = v_hist[b][:n].transpose(1, 0, 2)
     new_k = np.stack([k_hist[b][cache_lens[b]:] for b in range(B)])
@@ -188,8 +201,8 @@ def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11):
     po = torch.empty((num_splits, rows, d), dtype=torch.float32, device="cuda")
     pl = torch.empty((num_splits, rows), dtype=torch.float32, device="cuda")
     G.gemma_attn_decode(p, dev_bf16(q), dev_bf16(new_k), None if new_v is None else dev_bf16(new_v), dev_bf16(kc),
-                        None if vc is None else dev_bf16(vc), layout, cap, dev_i32(cache_lens), B, n_q, max_len,
-                        po, pl, num_splits)
+                        None if vc is None else dev_bf16(vc), layout | (G.CACHE_KEYS_ROTATED if keys_rotated else 0),
+                        cap, dev_i32(cache_lens), B, n_q, max_len, po, pl, num_splits)
     out = torch.empty((B, n_q, Hq, d), dtype=torch.float32, device="cuda")
     out16 = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
@@ -214,6 +227,15 @@ GLO = W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.25, rope_base=1e6)
 ])
 def test_decode_local_ring(cache_lens, n_q, splits):
     _check_decode(LOC, cache_lens, n_q, G.CACHE_RING, splits)
+
+
+@pytest.mark.parametrize("cache_lens,n_q,splits,layout", [
+    ((0, 5, 63, 64, 200), 1, None, G.CACHE_RING),       # warp kernel, split key / value stages
+    ((77, 300), 4, 3, G.CACHE_RING),                    # 8 rows per KV head
+    ((40, 150), 8, 2, G.CACHE_CONTIGUOUS),              # 16 rows: the CTA-wide kernel
+])
+def test_decode_local_prerotated_keys(cache_lens, n_q, splits, layout):
+    _check_decode(LOC, cache_lens, n_q, layout, splits, keys_rotated=True)
 
 
 def test_decode_local_contiguous():
