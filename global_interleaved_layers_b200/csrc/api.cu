@@ -224,6 +224,9 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
   a.window = global ? 0 : params->window; a.softmax_scale = params->softmax_scale; a.rot_mask = L.mask;
   a.out_f32 = params->out_dtype == GEMMA_ATTN_OUT_F32;
   a.pair_allowed = pair_kernel_enabled();
+  // 32-byte stores need the base and the row stride (head_dim elements) 32-byte aligned
+  a.out_align32 = ((reinterpret_cast<uintptr_t>(out) & 31u) == 0 &&
+                   (d * (a.out_f32 ? 4 : 2)) % 32 == 0) ? 1 : 0;
   cudaError_t e;
   switch (L.kd) {
     case 64: e = launch_prefill<64>(maps, a, stream); break;

@@ -23,6 +23,7 @@ struct PrefillArgs {
   float softmax_scale;
   int out_f32;        // 1: write fp32 output, 0: bf16
   int pair_allowed;   // 1: use the two-CTA paired kernel where the shape permits
+  int out_align32;    // 1: every output row segment is 32-byte aligned (256-bit stores)
   uint32_t rot_mask;  // bit c set: key/query chunk c (64 dims) is read from the rotated side copy
 };
 

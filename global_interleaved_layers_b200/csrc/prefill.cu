@@ -564,20 +564,33 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           const int col = c * 64 + h * 32;
           const uint32_t* oh = o + h * 32;
           if (valid && w.vpart * Cfg::kDv + col < args.head_dim) {
+            // a row segment of 32 columns: 128 bytes (f32) or 64 bytes (bf16), written with
+            // 32-byte stores where the output is 32-byte aligned (half the store
+            // instructions of 16-byte ones), else 16-byte stores
+            uint32_t wd[32];
+            int nw;
             if (args.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out) + obase + col);
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(oh[4 * i]) * inv_l, __uint_as_float(oh[4 * i + 1]) * inv_l,
-                                     __uint_as_float(oh[4 * i + 2]) * inv_l, __uint_as_float(oh[4 * i + 3]) * inv_l);
+              for (int i = 0; i < 32; ++i) wd[i] = __float_as_uint(__uint_as_float(oh[i]) * inv_l);
+              nw = 32;
             } else {
-              uint32_t wd[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 wd[i] = pack_bf16x2(__uint_as_float(oh[2 * i]) * inv_l, __uint_as_float(oh[2 * i + 1]) * inv_l);
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.out) + obase + col);
+              nw = 16;
+            }
+            uint8_t* dst = reinterpret_cast<uint8_t*>(args.out) + (obase + col) * (args.out_f32 ? 4 : 2);
+            if (args.out_align32) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+              for (int i = 0; i < 4; ++i)
+                if (8 * i < nw)
+                  st_global_32B(dst + 32 * i, make_uint4(wd[8 * i], wd[8 * i + 1], wd[8 * i + 2], wd[8 * i + 3]),
+                                make_uint4(wd[8 * i + 4], wd[8 * i + 5], wd[8 * i + 6], wd[8 * i + 7]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (4 * i < nw)
+                  *reinterpret_cast<uint4*>(dst + 16 * i) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
             }
           }
         }

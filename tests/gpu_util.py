@@ -51,7 +51,8 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     return W.bf16_bits_to_f32(W.f32_to_bf16_bits(np.asarray(x, dtype=np.float32)))
 
 
-def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=True, out_f32=False):
+def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=True, out_f32=False,
+                out_offset_bytes=0):
     """q/k/v: bf16 bit arrays (host) or bf16 device tensors. Returns (out device tensor, lse device).
 
     out is bf16 unless out_f32 (then float32, the accumulator precision)."""
@@ -65,7 +66,13 @@ def run_prefill(G, layer: W.LayerSpec, q, k, v, positions, cu_seqlens, with_lse=
     p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
                  rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale,
                  out_dtype=G.OUT_F32 if out_f32 else G.OUT_BF16)
-    out = torch.empty(qd.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    odt = torch.float32 if out_f32 else torch.bfloat16
+    if out_offset_bytes:  # an output that is only 16-byte aligned
+        esz = 4 if out_f32 else 2
+        extra = out_offset_bytes // esz
+        out = torch.empty((qd.numel() + extra,), dtype=odt, device="cuda")[extra:].view(qd.shape)
+    else:
+        out = torch.empty(qd.shape, dtype=odt, device="cuda")
     lse = torch.empty((Hq, T), dtype=torch.float32, device="cuda") if with_lse else None
     ws_bytes = G.gemma_attn_prefill_workspace_size(p, T)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")

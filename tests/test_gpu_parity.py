@@ -130,6 +130,20 @@ def test_prefill_shapes(layer, lens):
     _check_prefill(layer, lens, seed=3)
 
 
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_prefill_output_only_16_byte_aligned(out_f32):
+    # 32-byte output stores are used only where the output allows them; a 16-byte aligned
+    # output takes 16-byte stores and gives the same values
+    layer = W.LayerSpec(W.LOCAL, 4, 2, 256, window=100, rope_p=1.0, rope_base=1e4)
+    q, k, v = W.layer_inputs(layer, 300, 8)
+    cu = np.array([0, 300], np.int32)
+    pos = np.arange(300, dtype=np.int32)
+    a, _ = run_prefill(G, layer, q, k, v, pos, cu, out_f32=out_f32)
+    b, _ = run_prefill(G, layer, q, k, v, pos, cu, out_f32=out_f32, out_offset_bytes=16)
+    assert b.data_ptr() % 32 == 16
+    assert torch.equal(a, b)
+
+
 def test_prefill_position_offset():
     layer = W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
     _check_prefill(layer, (300,), seed=4, pos_start=100000)
