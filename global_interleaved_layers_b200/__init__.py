@@ -63,6 +63,8 @@ _lib.gemma_attn_last_launch_count.argtypes = []
 _lib.gemma_attn_last_launch_count.restype = ctypes.c_int
 _lib.gemma_attn_prefill_workspace_size.argtypes = [_PP, _I, ctypes.POINTER(ctypes.c_size_t)]
 _lib.gemma_attn_prefill.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
+_lib.gemma_attn_prefill_rotate.argtypes = _lib.gemma_attn_prefill.argtypes
+_lib.gemma_attn_prefill_attend.argtypes = _lib.gemma_attn_prefill.argtypes
 _lib.gemma_attn_decode.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _I, _P]
 _lib.gemma_attn_decode_num_splits.argtypes = [_PP, _I, _I, _I, ctypes.POINTER(ctypes.c_int32)]
 _lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
@@ -73,7 +75,8 @@ _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
 _lib.gemma_attn_selftest_timeout.argtypes = [_P, _P]
 for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_attn_decode",
            "gemma_attn_decode_num_splits", "gemma_attn_combine", "gemma_attn_tile_plan", "gemma_attn_check",
-           "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc", "gemma_attn_selftest_timeout"):
+           "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc", "gemma_attn_selftest_timeout",
+           "gemma_attn_prefill_rotate", "gemma_attn_prefill_attend"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -135,6 +138,24 @@ def gemma_attn_prefill(p: GemmaAttnParams, q, k, v, out, lse, positions, cu_seql
     _check(_lib.gemma_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                    _ptr(positions), _ptr(cu_seqlens), num_seqs, total_tokens, max_seqlen,
                                    _ptr(workspace), workspace_bytes, _stream(stream)), "gemma_attn_prefill")
+
+
+def gemma_attn_prefill_rotate(p: GemmaAttnParams, q, k, v, out, lse, positions, cu_seqlens, num_seqs: int,
+                              total_tokens: int, max_seqlen: int, workspace, workspace_bytes: int,
+                              stream=None) -> None:
+    _check(_lib.gemma_attn_prefill_rotate(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                          _ptr(positions), _ptr(cu_seqlens), num_seqs, total_tokens, max_seqlen,
+                                          _ptr(workspace), workspace_bytes, _stream(stream)),
+           "gemma_attn_prefill_rotate")
+
+
+def gemma_attn_prefill_attend(p: GemmaAttnParams, q, k, v, out, lse, positions, cu_seqlens, num_seqs: int,
+                              total_tokens: int, max_seqlen: int, workspace, workspace_bytes: int,
+                              stream=None) -> None:
+    _check(_lib.gemma_attn_prefill_attend(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                          _ptr(positions), _ptr(cu_seqlens), num_seqs, total_tokens, max_seqlen,
+                                          _ptr(workspace), workspace_bytes, _stream(stream)),
+           "gemma_attn_prefill_attend")
 
 
 def gemma_attn_decode(p: GemmaAttnParams, q, new_k, new_v, k_cache, v_cache, cache_layout: int,

@@ -147,10 +147,17 @@ int gemma_attn_prefill_workspace_size(const gemma_attn_params* params, int32_t t
   return GEMMA_ATTN_OK;
 }
 
-int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const void* k, const void* v, void* out,
-                       float* lse, const int32_t* positions, const int32_t* cu_seqlens, int32_t num_seqs,
-                       int32_t total_tokens, int32_t max_seqlen, void* workspace, size_t workspace_bytes,
-                       void* stream_) {
+}  // extern "C"
+
+namespace {
+enum : int { kPhaseRotate = 1, kPhaseAttend = 2 };
+
+// Prefill in two phases: the rotated side copies into the workspace, then the attention
+// kernel that reads them. gemma_attn_prefill runs both; the split entry points run one.
+int prefill_phases(const gemma_attn_params* params, const void* q, const void* k, const void* v, void* out,
+                   float* lse, const int32_t* positions, const int32_t* cu_seqlens, int32_t num_seqs,
+                   int32_t total_tokens, int32_t max_seqlen, void* workspace, size_t workspace_bytes,
+                   void* stream_, int phases) {
   t_launches = 0;
   int rc = check_params(params);
   if (rc != GEMMA_ATTN_OK) return rc;
@@ -173,10 +180,16 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
   uint16_t* vpad = reinterpret_cast<uint16_t*>(ws + L.v_off);
   const double log2_base = log2((double)params->rope_base);
 
-  if (L.mask) {
+  if (L.mask && (phases & kPhaseRotate)) {
     RopeArgs ra;
     ra.positions = positions; ra.tokens = total_tokens; ra.d = d; ra.r = L.r; ra.chunk_mask = L.mask;
     ra.n_out = L.n_out; ra.log2_base = log2_base;
+    // groups of 8 pairs (j, j + d/2) with a dim in a copied chunk: a prefix of the d/16 groups
+    ra.groups_active = 0;
+    for (int g = 0; g < d / 16; ++g) {
+      const int c0 = (8 * g) / 64, c1 = (8 * g + d / 2) / 64;
+      if (((L.mask >> c0) & 1u) || ((L.mask >> c1) & 1u)) ra.groups_active = g + 1;
+    }
     // queries and keys in one launch (the angles of a token serve both)
     ra.src = static_cast<const uint16_t*>(q); ra.dst = qside; ra.heads = Hq;
     ra.src2 = static_cast<const uint16_t*>(k); ra.dst2 = kside; ra.heads2 = Hkv;
@@ -189,6 +202,8 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
       ++t_launches;
     }
   }
+
+  if (!(phases & kPhaseAttend)) return GEMMA_ATTN_OK;
 
   PrefillMaps maps;
   bool ok = true;
@@ -238,6 +253,33 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
   if (e != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
   ++t_launches;
   return GEMMA_ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const void* k, const void* v, void* out,
+                       float* lse, const int32_t* positions, const int32_t* cu_seqlens, int32_t num_seqs,
+                       int32_t total_tokens, int32_t max_seqlen, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return prefill_phases(params, q, k, v, out, lse, positions, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                        workspace, workspace_bytes, stream, kPhaseRotate | kPhaseAttend);
+}
+
+int gemma_attn_prefill_rotate(const gemma_attn_params* params, const void* q, const void* k, const void* v,
+                              void* out, float* lse, const int32_t* positions, const int32_t* cu_seqlens,
+                              int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return prefill_phases(params, q, k, v, out, lse, positions, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                        workspace, workspace_bytes, stream, kPhaseRotate);
+}
+
+int gemma_attn_prefill_attend(const gemma_attn_params* params, const void* q, const void* k, const void* v,
+                              void* out, float* lse, const int32_t* positions, const int32_t* cu_seqlens,
+                              int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return prefill_phases(params, q, k, v, out, lse, positions, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                        workspace, workspace_bytes, stream, kPhaseAttend);
 }
 
 int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,

@@ -49,6 +49,7 @@ struct RopeArgs {
   int r;                    // rotated pairs (0: copy only)
   uint32_t chunk_mask;      // chunks of the (padded) head dim that are copied
   int n_out;
+  int groups_active;        // leading groups of 8 pairs with any dim in the copy (the rest: none)
   double log2_base;
 };
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream);

@@ -79,13 +79,15 @@ __device__ __forceinline__ void rope_heads(const uint16_t* __restrict__ src, uin
 // j0.. and j0 + d/2 ..).
 __global__ void rope_side_kernel(RopeArgs a) {
   const int half = a.d / 2;
-  const int groups = half / 8;
+  const int groups = a.groups_active;  // later groups have no dim in the copied chunks
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)a.tokens * groups) return;
   const int tok = (int)(idx / groups);
   const int j0 = (int)(idx % groups) * 8;
   const int col0 = side_col(a.chunk_mask, j0);
   const int col1 = side_col(a.chunk_mask, j0 + half);
+  const bool pad = a.d < 64 && j0 == 0;  // this thread also zeroes the padding columns d .. 63
+  if (col0 < 0 && col1 < 0 && !pad) return;  // neither half of these pairs is in the copy
   float c[8], s[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -93,13 +95,12 @@ __global__ void rope_side_kernel(RopeArgs a) {
     s[e] = 0.f;
     if (j0 + e < a.r) rope_cos_sin((double)a.positions[tok], rope_inv_freq_turns(j0 + e, a.d, a.log2_base), &c[e], &s[e]);
   }
-  const bool pad = a.d < 64 && j0 == 0;  // this thread also zeroes the padding columns d .. 63
   rope_heads(a.src, a.dst, a.heads, tok, a.d, a.n_out, j0, col0, col1, pad, c, s);
   if (a.heads2 > 0) rope_heads(a.src2, a.dst2, a.heads2, tok, a.d, a.n_out, j0, col0, col1, pad, c, s);
 }
 
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream) {
-  const long long total = (long long)a.tokens * (a.d / 16);
+  const long long total = (long long)a.tokens * a.groups_active;
   if (total == 0 || a.n_out == 0) return cudaSuccess;
   const int threads = 128;
   const long long blocks = (total + threads - 1) / threads;

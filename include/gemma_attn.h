@@ -126,6 +126,25 @@ int gemma_attn_prefill(const gemma_attn_params* params, const void* q, const voi
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The two phases of gemma_attn_prefill, for callers that schedule or time them apart:
+ * _rotate writes the rotated side copies of q and k (and, for head_dim < 64, the padded
+ * copies) into the workspace; _attend runs the attention kernel, which reads them, so it
+ * must follow a _rotate of the same q, k, v, positions and workspace on the same stream
+ * (or be otherwise ordered after it). Arguments, validation and errors are those of
+ * gemma_attn_prefill; _rotate ignores out, lse, cu_seqlens' contents and max_seqlen
+ * beyond validation. ("Visual guide to Gemma 4", section "p-RoPE": the rotation; the rest
+ * as gemma_attn_prefill.)
+ */
+int gemma_attn_prefill_rotate(const gemma_attn_params* params, const void* q, const void* k,
+                              const void* v, void* out, float* lse, const int32_t* positions,
+                              const int32_t* cu_seqlens, int32_t num_seqs, int32_t total_tokens,
+                              int32_t max_seqlen, void* workspace, size_t workspace_bytes, void* stream);
+int gemma_attn_prefill_attend(const gemma_attn_params* params, const void* q, const void* k,
+                              const void* v, void* out, float* lse, const int32_t* positions,
+                              const int32_t* cu_seqlens, int32_t num_seqs, int32_t total_tokens,
+                              int32_t max_seqlen, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode / speculative verify, split-KV stage: n_q new query tokens per sequence
  * attend to that sequence's cache plus the new tokens themselves.
  *   q          [batch, n_q, num_q_heads, head_dim] bf16; query i of sequence b sits at

@@ -144,6 +144,25 @@ def test_prefill_output_only_16_byte_aligned(out_f32):
     assert torch.equal(a, b)
 
 
+def test_prefill_rotate_then_attend_equals_prefill():
+    layer = W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
+    T = 400
+    q, k, _ = W.layer_inputs(layer, T, 12)
+    full, _ = run_prefill(G, layer, q, k, None, np.arange(T, dtype=np.int32), np.array([0, T], np.int32))
+    p = G.params(layer.kind, 8, 1, 512, rope_p=0.25, rope_base=1e6, softmax_scale=layer.softmax_scale)
+    ws_bytes = G.gemma_attn_prefill_workspace_size(p, T)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, 8, 512), dtype=torch.bfloat16, device="cuda")
+    args = (dev_bf16(q), dev_bf16(k), None, out, None, dev_i32(np.arange(T)), dev_i32(np.array([0, T])), 1, T, T,
+            ws, ws_bytes)
+    G.gemma_attn_prefill_rotate(p, *args)
+    assert G.gemma_attn_last_launch_count() == 1
+    G.gemma_attn_prefill_attend(p, *args)
+    assert G.gemma_attn_last_launch_count() == 1
+    G.gemma_attn_check()
+    assert torch.equal(out, full)
+
+
 def test_prefill_position_offset():
     layer = W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
     _check_prefill(layer, (300,), seed=4, pos_start=100000)
