@@ -36,7 +36,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of prefill_kernel<512> on the E2B global layer, from the
 # ncu capture summarised in profiles/prefill_kernel_d512_e2b_global.md. Reported only while the
 # kernel's sources still hash to the captured state; any change makes it null until re-captured.
-NCU_TRAFFIC = {"bytes": 103432960, "sources_sha256_16": "9cd34cebe70db882",
+NCU_TRAFFIC = {"bytes": 111479552, "sources_sha256_16": "6ef927675da9c7db",
                "sources": ["global_interleaved_layers_b200/csrc/prefill.cu",
                            "global_interleaved_layers_b200/csrc/common.cuh",
                            "global_interleaved_layers_b200/csrc/tile_plan.h",
@@ -640,7 +640,8 @@ def run_case(args):
         B, n_q, ctx = wl.batch, wl.n_q, (args.ctx or wl.cache_lens[0])
         Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
         cap = ctx if layer.k_eq_v else layer.window
-        layout = G.CACHE_CONTIGUOUS if layer.k_eq_v else G.CACHE_RING
+        # local: the serving layout with keys stored rotated (what per_kind.local_decode times)
+        layout = G.CACHE_CONTIGUOUS if layer.k_eq_v else (G.CACHE_RING | G.CACHE_KEYS_ROTATED)
         kc = torch.empty((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev).normal_(generator=gen)
         vc = None if layer.k_eq_v else torch.empty_like(kc).normal_(generator=gen)
         q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
