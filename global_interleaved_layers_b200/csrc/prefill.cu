@@ -47,7 +47,8 @@ constexpr int kBN = 128;
 constexpr int kChunk = 64;                   // dims per TMA box / swizzle row
 constexpr int kChunkBytes = 16384;           // 128 rows x 64 dims of bf16: a Q chunk or a V chunk
 constexpr int kMaxStages = 16;
-constexpr int kThreads = 192;
+constexpr int kBarrierBytes = 2048;           // mbarriers, TMEM base, softmax exchange
+constexpr int kThreads = 320;           // producer, MMA issuer, 8 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
@@ -71,10 +72,10 @@ struct PrefillCfg {
   static constexpr int kKStages = kQChunks / kKPerStage;
   static constexpr int kVStages = (PAIR ? kVChunks / 2 : kVChunks) / kVPerStage;
   static constexpr int kPvN = (PAIR ? 2 : 1) * kVPerStage * kChunk;  // output columns per V stage
-  static constexpr int kRingBudget = 232448 - 1024 /*align*/ - 512 /*barriers*/ - kQBytes;
+  static constexpr int kRingBudget = 232448 - 1024 /*align*/ - kBarrierBytes - kQBytes;
   static constexpr int kStages = kRingBudget / kStageBytes < kMaxStages ? kRingBudget / kStageBytes : kMaxStages;
   static constexpr int kSmemData = kQBytes + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int kSmemBytes = kSmemData + 1024 /*align*/ + kBarrierBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(!PAIR || D >= 128, "paired form needs at least two 64-dim chunks");
   static_assert(kKStages >= 1 && kVStages >= 1 && kStages >= 2, "ring shape");
@@ -94,7 +95,11 @@ struct __align__(8) Barriers {
   uint64_t ring_empty[kMaxStages];
   uint32_t tmem_base;
   int abort_flag;
+  uint64_t xfull[4];   // per TMEM lane quadrant: both halves wrote their exchange values
+  uint64_t xfree[4];   // per quadrant: both halves read them (the slots may be rewritten)
+  float xch[2 * 128];  // softmax half-row exchange: [half][row] tile maxima, then row sums
 };
+static_assert(sizeof(Barriers) <= kBarrierBytes, "barrier block");
 
 // 2^x on the SFU (ex2.approx, flush-to-zero): P is rounded to bf16 and the row sums
 // carry far more error than the approximation's few ulp.
@@ -190,12 +195,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     mbar_init(&bars->q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], PAIR ? 8 : 4);  // one arrival per softmax warp (of both CTAs)
+      mbar_init(&bars->p_full[b], PAIR ? 16 : 8);  // one arrival per softmax warp (of both CTAs)
     }
     mbar_init(&bars->pv_done[0], 1);
     mbar_init(&bars->pv_done[1], 1);
     mbar_init(&bars->o_ready, 1);
-    mbar_init(&bars->o_empty, PAIR ? 8 : 4);
+    mbar_init(&bars->o_empty, PAIR ? 16 : 8);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars->xfull[q], 2);
+      mbar_init(&bars->xfree[q], 2);
+    }
     mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&bars->ring_full[s], load_arrivals);
@@ -430,10 +439,37 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Eight warps: warps w and w + 4 share the TMEM lane quadrant w % 4 (rows quad*32 ..
+    // +31, one row per lane) and split each score tile's 128 columns, half h taking
+    // columns 64h .. 64h + 63 (and O columns h*kDv/2 ..). The two halves of a row agree on
+    // the tile maximum through a shared-memory slot per row and half, handed over with two
+    // bounded mbarriers per quadrant (written / read); row sums are combined once, at the
+    // epilogue. Both halves run the same exchanges in the same order, so the exchange
+    // count x gives both barriers' phase.
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float scale_log2 = args.softmax_scale * 1.4426950408889634f;
+    constexpr int kHC = kBN / 2;               // score columns per half
+    constexpr int kHO = Cfg::kDv / 2;          // output columns per half
+    float* xch = bars->xch;                    // [2 halves][128 rows]
+    uint32_t xk = 0;                           // exchanges so far (both halves alike)
+    // Publish v for this row and return the partner half's value (ok = false on abort).
+    auto exchange = [&](float v, bool& okx) -> float {
+      xch[half * kBM + row] = v;
+      tc_fence_before();  // this half's score loads are ordered before the arrival
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->xfull[quad]);
+      okx = __all_sync(0xffffffffu, mbar_wait(&bars->xfull[quad], xk & 1u, abort_flag));
+      tc_fence_after();
+      const float other = okx ? xch[(1 - half) * kBM + row] : v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->xfree[quad]);
+      if (okx) okx = __all_sync(0xffffffffu, mbar_wait(&bars->xfree[quad], xk & 1u, abort_flag));
+      ++xk;
+      return other;
+    };
     bool ok = true;
     int g = 0;
     int unit_iter = 0;
@@ -441,19 +477,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       Unit w;
       if (!unit_of_round(r, w)) continue;
       float m_used = -INFINITY;
-      float l_sum = 0.f;
+      float l_part = 0.f;
       const int grow = w.row0 + row;  // in-sequence offset of this thread's query row
       for (int jj = 0; jj < w.ntiles && ok; ++jj) {
         const int t = g + jj;
         const int b = t & 1;
-        const uint32_t s_col = b ? kColS1 : kColS0;
+        const uint32_t s_col = (b ? kColS1 : kColS0) + half * kHC;
         ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->s_full[b], (uint32_t)(t >> 1) & 1u, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        float sv[kBN];
+        float sv[kHC];
         uint32_t* tr = reinterpret_cast<uint32_t*>(sv);
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
+        for (int c = 0; c < kHC / 32; ++c) tmem_ld_x32(tmem + lane_off + s_col + c * 32, tr + c * 32);
         tmem_ld_wait();
         const int kt = w.kt_lo + jj;
         // A key tile that runs past the end of the sequence holds the next sequence's
@@ -462,14 +498,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
                              kv_tile_class(is_local, args.window, w.len, w.qt, kt, kBM, kBN) != kTileFull;
         // Masked tiles are scaled here (masked entries -inf); full tiles keep raw scores and
         // fold the scale into the exponent's FFMA (scale > 0, so the max commutes with it).
-        // Eight partial maxima keep the reduction off one long dependency chain.
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
         if (partial) {
-          const int k0 = kt * kBN;
+          const int k0 = kt * kBN + half * kHC;
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
+          for (int c = 0; c < kHC; ++c) {
             const int key = k0 + c;
             const bool vis = key <= grow && (!is_local || key > grow - args.window);
             sv[c] = vis ? sv[c] * scale_log2 : -INFINITY;
@@ -477,12 +512,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+          for (int c = 0; c < kHC; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
         }
         const float coef = partial ? 1.f : scale_log2;
-        float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+        float m_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        if (!partial) m_tile *= scale_log2;
+        if (!partial) m_half *= scale_log2;
+        // the row's tile maximum: both halves take the max of the same two values (this
+        // also orders both halves' score loads before either writes its P below)
+        const float m_tile = fmaxf(m_half, exchange(m_half, ok));
+        if (!ok) break;
         // Raise the running max only when it grows by more than 2^8 (or was empty); P
         // may then exceed 1 by up to 2^8, which fp32 sums and bf16 P absorb.
         float alpha = 1.f;
@@ -490,7 +529,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         if (m_tile > m_used + kRescaleThreshold || (m_used == -INFINITY && m_tile > -INFINITY)) {
           if (m_used != -INFINITY) {
             alpha = fast_exp2(m_used - m_tile);
-            l_sum *= alpha;
+            l_part *= alpha;
             rescale_o = true;
           }
           m_used = m_tile;
@@ -498,25 +537,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         // P(t) goes over S(t) right away: that buffer's previous P (tile t-2) was consumed
         // by PV(t-2), which finished before S(t) was computed.
         const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-        uint32_t p[kBN / 2];
+        uint32_t p[kHC / 2];
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kBN / 2; ++c) {
+        for (int c = 0; c < kHC / 2; ++c) {
           const float p0 = fast_exp2(fmaf(sv[2 * c], coef, -m_sub));
           const float p1 = fast_exp2(fmaf(sv[2 * c + 1], coef, -m_sub));
           rs4[c & 3] += p0 + p1;
           p[c] = pack_bf16x2(p0, p1);
         }
-        l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-        tmem_st_x32(tmem + lane_off + s_col, p);
-        tmem_st_x32(tmem + lane_off + s_col + 32, p + 32);
-        // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any
-        // lane needs it, each lane with its own factor (1 for lanes that do not). O may only
-        // be touched once PV(t-1) has finished; without a rescale the warp does not wait,
-        // since PV(t) is issued after PV(t-1) and the tensor core runs them in order. The
-        // parity wait is exact: PV(t-3) finished before S(t-1) was issued, and PV(t+1) needs
-        // this warp's p_full(t+1) arrival, so PV(t-1) is the only phase of its barrier that
-        // can still be pending. A unit's first tile never rescales (m_used starts empty).
+        l_part += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        // this half's P: TMEM columns (tile base) + 32 half .. + 31 (two bf16 per column)
+        tmem_st_x32(tmem + lane_off + (b ? kColS1 : kColS0) + half * (kHC / 2), p);
+        // tcgen05.ld/st are warp-collective: the warp rescales its half of the O rows together
+        // when any lane needs it, each lane with its own factor (1 for lanes that do not). O
+        // may only be touched once PV(t-1) has finished; without a rescale the warp does not
+        // wait, since PV(t) is issued after PV(t-1) and the tensor core runs them in order.
+        // The parity wait is exact: PV(t-3) finished before S(t-1) was issued, and PV(t+1)
+        // needs this warp's p_full(t+1) arrival, so PV(t-1) is the only phase of its barrier
+        // that can still be pending. A unit's first tile never rescales (m_used starts empty).
         const bool rescale_warp = __any_sync(0xffffffffu, rescale_o);
         if (rescale_warp && jj >= 1) {
           ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->pv_done[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag));
@@ -528,13 +567,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         }
         if (rescale_warp) {
 #pragma unroll 1
-          for (int c = 0; c < Cfg::kDv / 32; ++c) {
+          for (int c = 0; c < kHO / 32; ++c) {
             uint32_t o[32];
-            tmem_ld_x32(tmem + lane_off + kColO + c * 32, o);
+            tmem_ld_x32(tmem + lane_off + kColO + half * kHO + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(tmem + lane_off + kColO + c * 32, o);
+            tmem_st_x32(tmem + lane_off + kColO + half * kHO + c * 32, o);
           }
         }
         tmem_st_wait();
@@ -546,6 +585,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         }
       }
       if (!ok) break;
+      // the row sum: this half's part plus the partner half's
+      const float l_sum = l_part + exchange(l_part, ok);
+      if (!ok) break;
       ok = __all_sync(0xffffffffu, wait_bar<PAIR>(&bars->o_ready, (uint32_t)unit_iter & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -554,48 +596,43 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       const int tok = w.tok0 + grow;
       const size_t obase = ((size_t)tok * args.num_q_heads + w.head) * args.head_dim + w.vpart * Cfg::kDv;
 #pragma unroll 1
-      for (int c = 0; c < Cfg::kDv / 64; ++c) {
-        uint32_t o[64];
-        tmem_ld_x32(tmem + lane_off + kColO + c * 64, o);
-        tmem_ld_x32(tmem + lane_off + kColO + c * 64 + 32, o + 32);
+      for (int c = 0; c < kHO / 32; ++c) {
+        uint32_t oh[32];
+        tmem_ld_x32(tmem + lane_off + kColO + half * kHO + c * 32, oh);
         tmem_ld_wait();
+        const int col = half * kHO + c * 32;
+        if (valid && w.vpart * Cfg::kDv + col < args.head_dim) {
+          // a row segment of 32 columns: 128 bytes (f32) or 64 bytes (bf16), written with
+          // 32-byte stores where the output is 32-byte aligned (half the store
+          // instructions of 16-byte ones), else 16-byte stores
+          uint32_t wd[32];
+          int nw;
+          if (args.out_f32) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col = c * 64 + h * 32;
-          const uint32_t* oh = o + h * 32;
-          if (valid && w.vpart * Cfg::kDv + col < args.head_dim) {
-            // a row segment of 32 columns: 128 bytes (f32) or 64 bytes (bf16), written with
-            // 32-byte stores where the output is 32-byte aligned (half the store
-            // instructions of 16-byte ones), else 16-byte stores
-            uint32_t wd[32];
-            int nw;
-            if (args.out_f32) {
+            for (int i = 0; i < 32; ++i) wd[i] = __float_as_uint(__uint_as_float(oh[i]) * inv_l);
+            nw = 32;
+          } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) wd[i] = __float_as_uint(__uint_as_float(oh[i]) * inv_l);
-              nw = 32;
-            } else {
+            for (int i = 0; i < 16; ++i)
+              wd[i] = pack_bf16x2(__uint_as_float(oh[2 * i]) * inv_l, __uint_as_float(oh[2 * i + 1]) * inv_l);
+            nw = 16;
+          }
+          uint8_t* dst = reinterpret_cast<uint8_t*>(args.out) + (obase + col) * (args.out_f32 ? 4 : 2);
+          if (args.out_align32) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                wd[i] = pack_bf16x2(__uint_as_float(oh[2 * i]) * inv_l, __uint_as_float(oh[2 * i + 1]) * inv_l);
-              nw = 16;
-            }
-            uint8_t* dst = reinterpret_cast<uint8_t*>(args.out) + (obase + col) * (args.out_f32 ? 4 : 2);
-            if (args.out_align32) {
+            for (int i = 0; i < 4; ++i)
+              if (8 * i < nw)
+                st_global_32B(dst + 32 * i, make_uint4(wd[8 * i], wd[8 * i + 1], wd[8 * i + 2], wd[8 * i + 3]),
+                              make_uint4(wd[8 * i + 4], wd[8 * i + 5], wd[8 * i + 6], wd[8 * i + 7]));
+          } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (8 * i < nw)
-                  st_global_32B(dst + 32 * i, make_uint4(wd[8 * i], wd[8 * i + 1], wd[8 * i + 2], wd[8 * i + 3]),
-                                make_uint4(wd[8 * i + 4], wd[8 * i + 5], wd[8 * i + 6], wd[8 * i + 7]));
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                if (4 * i < nw)
-                  *reinterpret_cast<uint4*>(dst + 16 * i) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
-            }
+            for (int i = 0; i < 8; ++i)
+              if (4 * i < nw)
+                *reinterpret_cast<uint4*>(dst + 16 * i) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
           }
         }
       }
-      if (valid && w.vpart == 0 && args.lse != nullptr)
+      if (half == 0 && valid && w.vpart == 0 && args.lse != nullptr)
         args.lse[(size_t)w.head * args.total_tokens + tok] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
       // O has been read out: the next unit's first value MMA may overwrite it
       tc_fence_before();
