@@ -559,9 +559,23 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
         log(f"decode kind={layer.kind}")
 
         def measure(layout):
+            # one split: the one-call entry point, whose decode kernel writes the output itself;
+            # several: the split partials, then the combine
+            def dec():
+                if splits == 1:
+                    G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, 1, out,
+                                                None, stream)
+                else:
+                    G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits,
+                                        stream)
+
+            def comb():
+                if splits > 1:
+                    G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+
             def one():
-                G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
-                G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+                dec()
+                comb()
 
             for _ in range(args.warmup):
                 one()
@@ -576,9 +590,9 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
                 e1 = torch.cuda.Event(enable_timing=True)
                 e2 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+                dec()
                 e1.record(stream)
-                G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+                comb()
                 e2.record(stream)
                 evs.append((e0, e2))
                 dec_evs.append((e0, e1))
@@ -591,6 +605,7 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
             gbs = nbytes / (ms * 1e-3) / 1e9
             rotated = bool(layout & G.CACHE_KEYS_ROTATED)
             return {"gbs": gbs, "ms": ms, "decode_kernel_ms": dec_ms, "bytes": nbytes, "splits": splits,
+                    "launches": 1 if splits == 1 else 2,
                     "frac_of_hbm": gbs / peaks["hbm_gbs"],
                     "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} ctx={ctx} " + (
                         "K=V contiguous" if layer.k_eq_v else
@@ -657,8 +672,12 @@ def run_case(args):
         out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
 
         def op():
-            G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
-            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
+            if splits == 1:
+                G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, 1, out, None,
+                                            stream)
+            else:
+                G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, ctx, po, pl, splits, stream)
+                G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
     for _ in range(args.warmup + args.steps):
         op()
     torch.cuda.synchronize()

@@ -333,7 +333,7 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   if (group * n_q > decode_max_rows(params->head_dim)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
     return GEMMA_ATTN_ERR_MISALIGNED;
-  DecodeArgs a;
+  DecodeArgs a{};  // out == nullptr: the kernel writes the split partials
   a.q = static_cast<const uint16_t*>(q);
   a.new_k = static_cast<const uint16_t*>(new_k);
   a.new_v = static_cast<const uint16_t*>(new_v);

@@ -19,7 +19,9 @@
 //   3. S^T = K Q^T on tensor cores (mma.sync m16n8k16 bf16, keys on M, rows on N);
 //   4. online softmax per row across the 4 warps;
 //   5. O^T += V^T P^T on tensor cores, the warps splitting the head dim.
-// The CTA writes an fp32 partial (O / l) and its log-sum-exp for the combine.
+// The CTA writes an fp32 partial (O / l) and its log-sum-exp for the combine; with a
+// single split and a final output given, it writes that output and log-sum-exp
+// directly instead (the combine of one split is the identity).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -59,6 +61,23 @@ __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint
 __device__ __forceinline__ uint16_t f2bf(float f) {
   __nv_bfloat16 h = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// Result of one row element / one row: the split partial, or, in direct mode (one
+// split, a.out set), the final output element in the caller's dtype.
+__device__ __forceinline__ void put_o(const DecodeArgs& a, size_t i, float v) {
+  if (a.out == nullptr)
+    a.partial_o[i] = v;
+  else if (a.out_f32)
+    static_cast<float*>(a.out)[i] = v;
+  else
+    static_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ void put_lse(const DecodeArgs& a, size_t i, float v) {
+  if (a.out == nullptr)
+    a.partial_lse[i] = v;
+  else if (a.out_lse != nullptr)
+    a.out_lse[i] = v;
 }
 
 // Shared-memory carve-up of the decode kernel (element counts are bf16 unless noted).
@@ -474,16 +493,16 @@ decode_tc_kernel(DecodeArgs a) {
         const size_t orow = ((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh;
         const float l = l_run[nt][e];
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float* po = a.partial_o + ((size_t)split * rows_total + orow) * D;
+        const size_t po = ((size_t)split * rows_total + orow) * D;
 #pragma unroll
         for (int mt = 0; mt < MTW; ++mt) {
           const int d0 = (warp * MTW + mt) * 16;
-          po[d0 + g] = oacc[mt][nt][e] * inv;
-          po[d0 + g + 8] = oacc[mt][nt][2 + e] * inv;
+          put_o(a, po + d0 + g, oacc[mt][nt][e] * inv);
+          put_o(a, po + d0 + g + 8, oacc[mt][nt][2 + e] * inv);
         }
         if (warp == 0 && g == 0)
-          a.partial_lse[(size_t)split * rows_total + orow] =
-              l > 0.f ? (m_run[nt][e] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+          put_lse(a, (size_t)split * rows_total + orow,
+                  l > 0.f ? (m_run[nt][e] + log2f(l)) * 0.6931471805599453f : -INFINITY);
       }
   }
 }
@@ -997,13 +1016,13 @@ decode_warp_kernel(DecodeArgs a) {
 #pragma unroll
     for (int w = 0; w < kWWarps; ++w) acc += red[(size_t)(w * 8 + row) * L::RED + d];
     const size_t orow = ((size_t)b * a.n_q + row / group) * a.num_q_heads + kvh * group + row % group;
-    a.partial_o[((size_t)split * rows_total + orow) * D + d] = acc;
+    put_o(a, ((size_t)split * rows_total + orow) * D + d, acc);
   }
   if (tid < R) {
     float M, Lsum;
     merged(tid, M, Lsum);
     const size_t orow = ((size_t)b * a.n_q + tid / group) * a.num_q_heads + kvh * group + tid % group;
-    a.partial_lse[(size_t)split * rows_total + orow] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY;
+    put_lse(a, (size_t)split * rows_total + orow, Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY);
   }
 }
 

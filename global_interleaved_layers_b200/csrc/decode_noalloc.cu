@@ -10,6 +10,8 @@
 // Nothing in it needs clearing: every call rewrites all of the partials it reads.
 // Two calls that overlap on the GPU (different streams, or host threads without
 // ordering between their streams) race on it.
+// With num_splits == 1 there are no partials: the decode kernel writes the output and
+// log-sum-exp itself, in one launch, and the array is not touched.
 #include <atomic>
 #include <mutex>
 
@@ -94,19 +96,30 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
     return GEMMA_ATTN_ERR_MISALIGNED;
 
-  // Partials for num_splits x rows: fp32 O [splits, rows, d] then fp32 lse [splits, rows].
+  // One split: the decode kernel writes out and lse itself (the combine of a single
+  // partial is the identity) and nothing is staged. Otherwise partials for
+  // num_splits x rows: fp32 O [splits, rows, d] then fp32 lse [splits, rows].
+  const bool direct = num_splits == 1;
   const size_t rows = (size_t)batch * n_q * params->num_q_heads;
   const size_t o_bytes = align256((size_t)num_splits * rows * d * sizeof(float));
   const size_t l_bytes = align256((size_t)num_splits * rows * sizeof(float));
-  if (o_bytes + l_bytes > kNoAllocBytes) return GEMMA_ATTN_ERR_WORKSPACE;
+  float* partial_o = nullptr;
+  float* partial_lse = nullptr;
+  if (!direct) {
+    if (o_bytes + l_bytes > kNoAllocBytes) return GEMMA_ATTN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != GEMMA_ATTN_OK) return rc;
+    partial_o = static_cast<float*>(scratch);
+    partial_lse = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes);
+  }
 
-  void* scratch = nullptr;
-  const int rc = noalloc_scratch(&scratch);
-  if (rc != GEMMA_ATTN_OK) return rc;
-  float* partial_o = static_cast<float*>(scratch);
-  float* partial_lse = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes);
-
-  DecodeArgs a;
+  DecodeArgs a{};
+  if (direct) {
+    a.out = out;
+    a.out_lse = lse;
+    a.out_f32 = params->out_dtype == GEMMA_ATTN_OUT_F32;
+  }
   a.q = static_cast<const uint16_t*>(q);
   a.new_k = static_cast<const uint16_t*>(new_k);
   a.new_v = static_cast<const uint16_t*>(new_v);
@@ -125,6 +138,7 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
   if (!decode_supported(a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (launch_decode(a, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
+  if (direct) return GEMMA_ATTN_OK;
 
   CombineArgs c;
   c.partial_o = partial_o; c.partial_lse = partial_lse; c.out = out; c.lse = lse;

@@ -63,6 +63,9 @@ struct DecodeArgs {
   const int32_t* cache_seqlens;
   float* partial_o;         // [splits, rows, d]
   float* partial_lse;       // [splits, rows]
+  void* out;                // null: write the partials; else (num_splits == 1) the final [rows, d] output
+  float* out_lse;           // with out: final log-sum-exp [rows] or null
+  int out_f32;              // with out: 1 fp32, 0 bf16
   int batch, n_q, num_q_heads, num_kv_heads, head_dim;
   int is_local, window, ring, capacity, num_splits;
   int keys_rotated;         // cached keys are stored rotated: only new tokens' keys are rotated here

@@ -199,6 +199,8 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
  *   each call rewrites every partial it reads, so nothing is cleared between calls.
  *   Calls that overlap on the GPU (concurrent streams, or threads whose streams are
  *   not ordered) race on the array and corrupt each other's results.
+ *   num_splits == 1: the decode kernel writes out and lse itself (one launch); the
+ *   static array is neither used nor size-checked, and such calls do not race.
  */
 #define GEMMA_ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
 int gemma_attn_decode_noalloc(const gemma_attn_params* params, const void* q, const void* new_k,

@@ -82,3 +82,41 @@ def test_noalloc_rejects_requests_beyond_the_static_buffer():
         G.gemma_attn_decode_noalloc(p, fake, fake, None, fake, None, G.CACHE_CONTIGUOUS, 1000, fake, B, n_q, 1000,
                                     splits, fake, None)
     assert e.value.status == G.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("layer,cache_lens,n_q,ring,out_dtype", [
+    # 8 rows per KV head and 2 new tokens: 16 rows, the tensor-core split kernel
+    (W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.25, rope_base=1e6), (300, 1000), 2, False, "f32"),
+    # 2 rows per KV head: the warp-split kernel, bf16 output, keys stored rotated
+    (W.LayerSpec(W.LOCAL, 8, 4, 256, window=128, rope_p=1.0, rope_base=1e4), (50, 700), 1, True, "bf16"),
+    (W.LayerSpec(W.LOCAL, 8, 4, 256, window=128, rope_p=1.0, rope_base=1e4), (0, 129), 1, True, "f32"),
+])
+def test_noalloc_single_split_writes_the_combined_result_directly(layer, cache_lens, n_q, ring, out_dtype):
+    """One split: the decode kernel writes out and lse itself, bit for bit what the combine
+    of its single partial writes (exp(0) = 1 weights, division by 1)."""
+    B = len(cache_lens)
+    Hq, d = layer.num_q_heads, layer.head_dim
+    rows = B * n_q * Hq
+    layout = (G.CACHE_RING | G.CACHE_KEYS_ROTATED) if ring else G.CACHE_CONTIGUOUS
+    od = G.OUT_F32 if out_dtype == "f32" else G.OUT_BF16
+    tdt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    p = G.params(layer.kind, Hq, layer.num_kv_heads, d, window=layer.window, rope_p=layer.rope_p,
+                 rope_base=layer.rope_base, softmax_scale=layer.softmax_scale, out_dtype=od)
+    max_len = max(cache_lens)
+    lens = dev_i32(cache_lens)
+    q, nk, nv, kc, vc, cap = _inputs(layer, cache_lens, n_q, 43, ring)
+    po = torch.empty((1, rows, d), dtype=torch.float32, device="cuda")
+    pl = torch.empty((1, rows), dtype=torch.float32, device="cuda")
+    G.gemma_attn_decode(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, po, pl, 1)
+    ref = torch.empty((B, n_q, Hq, d), dtype=tdt, device="cuda")
+    ref_lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    G.gemma_attn_combine(po, pl, 1, rows, d, od, ref, ref_lse)
+    out = torch.full((B, n_q, Hq, d), float("nan"), dtype=tdt, device="cuda")
+    lse = torch.full((rows,), float("nan"), dtype=torch.float32, device="cuda")
+    G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, 1, out, lse)
+    out_nolse = torch.full_like(out, float("nan"))
+    G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, 1, out_nolse, None)
+    G.gemma_attn_check()
+    assert torch.equal(out, ref)
+    assert torch.equal(out_nolse, ref)
+    assert torch.equal(lse, ref_lse)
