@@ -316,9 +316,15 @@ def main():
         return reps.max_over_ranks(x, dev)
 
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def flush_l2():
+        # write 256 MiB (evicts every line of the previous step), then read another 256 MiB:
+        # the written lines leave L2 (written back) before the timed step, which then starts
+        # with L2 holding only clean lines of neither input nor output
         flush_buf.fill_(1.0)
+        torch.sum(flush_read, dtype=torch.float32, out=flush_sink)
 
     # ------------------------------------------------------------------ prefill block inputs
     wl = W.e2b_block()
@@ -494,7 +500,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "global_batch": 1, "seq_len": L,
                    "layers": "4 local (W=512, 8/4 heads, d=256) + 1 global (8/1 heads, d=512, K=V, p=0.25)",
-                   "l2": "flushed before every timed step (256 MiB write); per-step CUDA events",
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another "
+                          "buffer, so no dirty lines are left for the step to write back); per-step CUDA events",
                    "parallelism": f"replicas x{world}"},
         "per_kind": {
             "local_prefill": {"tflops": l_tflops, "ms": l_ms, "frac_of_peak": l_tflops / peak_t,

@@ -706,33 +706,42 @@ decode_warp_kernel(DecodeArgs a) {
     fence_barrier_init();
   }
   if (tid == 0) *abort_flag = 0;
-  __syncwarp();
-  // the first blocks stream in while the CTA prepares queries and angle tables
-  if constexpr (kSplit) {
-    for (int s = 0; s < kWStages && s < my_n; ++s) issue_half(s, 0);
-    for (int s = 0; s < NSV && s < my_n; ++s) issue_half(s, 1);
-  } else {
-    for (int s = 0; s < kWStages && s < my_n; ++s) issue(s);
-  }
 
-  // rotated queries (bf16); rows R..7 are zero
-  for (int idx = tid; idx < 8 * HALF; idx += kWWarps * 32) {
-    const int row = idx / HALF, j = idx % HALF;
-    float y0 = 0.f, y1 = 0.f;
+  // The query rows are loaded, and land, before this CTA issues any copy: queued behind
+  // the copies of the GPU's other CTAs (tens of MB at the start), a query load would
+  // hold up the start of the computation by microseconds.
+  constexpr int QCH = D / 8;  // 16-byte chunks per query row
+  constexpr int QV = (8 * QCH + NW * 32 - 1) / (NW * 32);
+#pragma unroll
+  for (int k = 0; k < QV; ++k) {
+    const int idx = tid + k * NW * 32;
+    const int row = idx / QCH;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
     if (row < R) {
       const int i = row / group, hh = row % group;
-      const uint16_t* qrow = a.q + (((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh) * D;
-      const float x0 = bf2f(qrow[j]), x1 = bf2f(qrow[j + HALF]);
-      y0 = x0; y1 = x1;
-      if (j < r) {
-        float c, s;
-        rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
-        y0 = x0 * c - x1 * s;
-        y1 = x0 * s + x1 * c;
-      }
+      x = *reinterpret_cast<const uint4*>(a.q + (((size_t)b * a.n_q + i) * a.num_q_heads + kvh * group + hh) * D +
+                                          (idx % QCH) * 8);
     }
-    qs[row * KST + j] = f2bf(y0);
-    qs[row * KST + j + HALF] = f2bf(y1);
+    if (idx < 8 * QCH) *reinterpret_cast<uint4*>(qs + row * KST + (idx % QCH) * 8) = x;  // rows R..7 zero
+  }
+  __syncthreads();
+  // Only the first block's key rows are copied now: a warp's issue of bulk copies stalls
+  // while the SM's copy queue is full, so the rest of the ring is issued at the top of
+  // the first iteration, behind the wait for these rows.
+  if constexpr (kSplit) {
+    if (my_n > 0) issue_half(0, 0);
+  } else {
+    if (my_n > 0) issue(0);
+  }
+  // the first r pairs of the query rows, rotated in place (bf16)
+  for (int idx = tid; idx < R * r; idx += kWWarps * 32) {
+    const int row = idx / r, j = idx % r;
+    const int i = row / group;
+    const float x0 = bf2f(qs[row * KST + j]), x1 = bf2f(qs[row * KST + j + HALF]);
+    float c, s;
+    rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
+    qs[row * KST + j] = f2bf(x0 * c - x1 * s);
+    qs[row * KST + j + HALF] = f2bf(x0 * s + x1 * c);
   }
   // per-pair frequencies (turns per position), cos / sin of theta_j (one key) and of
   // 16 NW theta_j (one block step of a warp); pairs past r get the identity
@@ -782,6 +791,14 @@ decode_warp_kernel(DecodeArgs a) {
   bool ok = true;
   for (; it < my_n; ++it) {
     const int st = it % kWStages;
+    if (it == 0) {  // the rest of the ring: the first value rows, then further key stages
+      if constexpr (kSplit) {
+        for (int s = 0; s < NSV && s < my_n; ++s) issue_half(s, 1);
+        for (int s = 1; s < kWStages && s < my_n; ++s) issue_half(s, 0);
+      } else {
+        for (int s = 1; s < kWStages && s < my_n; ++s) issue(s);
+      }
+    }
     ok = mbar_wait(&wbar[st], (uint32_t)(it / kWStages) & 1u, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;

@@ -297,6 +297,12 @@ def test_decode_global_gqa8():
     (W.LOCAL, 8, 4, 64, 0.75, 4),     # r = 24
     (W.LOCAL, 2, 2, 128, 0.3, 1),     # r = 19
     (W.LOCAL, 8, 1, 512, 1.0, 1),     # separate-V d = 512: one ring stage per warp
+    # up to 2 rows per KV head
+    (W.GLOBAL, 2, 1, 512, 0.25, 1),   # K=V, rotated k-steps read from the rotated copy
+    (W.GLOBAL, 1, 1, 128, 0.3, 1),    # one row, r = 19
+    (W.GLOBAL, 2, 1, 256, 1.0, 1),    # every k-step rotated
+    (W.LOCAL, 2, 1, 512, 1.0, 1),     # separate-V d = 512
+    (W.LOCAL, 1, 1, 256, 0.5, 2),     # 2 rows from 2 new tokens of one head
 ])
 def test_decode_head_dims_and_partial_rotation(kind, hq, hkv, d, p, n_q):
     window = 48 if kind == W.LOCAL else 0
