@@ -324,7 +324,7 @@ def main():
         # the written lines leave L2 (written back) before the timed step, which then starts
         # with L2 holding only clean lines of neither input nor output
         flush_buf.fill_(1.0)
-        torch.sum(flush_read, dtype=torch.float32, out=flush_sink)
+        torch.sum(flush_read, dim=0, out=flush_sink)
 
     # ------------------------------------------------------------------ prefill block inputs
     wl = W.e2b_block()

@@ -496,28 +496,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
         const bool partial = (kt + 1) * kBN > w.len ||
                              kv_tile_class(is_local, args.window, w.len, w.qt, kt, kBM, kBN) != kTileFull;
-        // Masked tiles are scaled here (masked entries -inf); full tiles keep raw scores and
-        // fold the scale into the exponent's FFMA (scale > 0, so the max commutes with it).
+        // Scores stay unscaled: the scale is folded into the exponent's FFMA (scale > 0, so
+        // the max commutes with it). In a masked tile the keys a row sees are one run of
+        // the half's columns, [c_lo, c_hi] (causal: key <= row; local: key > row - window;
+        // past the row's sequence end nothing, since row < len); the rest become -inf.
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
         if (partial) {
           const int k0 = kt * kBN + half * kHC;
+          const int c_hi = grow - k0;
+          const int c_lo = is_local ? grow - args.window + 1 - k0 : 0;
 #pragma unroll
           for (int c = 0; c < kHC; ++c) {
-            const int key = k0 + c;
-            const bool vis = key <= grow && (!is_local || key > grow - args.window);
-            sv[c] = vis ? sv[c] * scale_log2 : -INFINITY;
+            sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
             mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < kHC; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
         }
-        const float coef = partial ? 1.f : scale_log2;
-        float m_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        if (!partial) m_half *= scale_log2;
+        const float coef = scale_log2;
+        const float m_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
         // the row's tile maximum: both halves take the max of the same two values (this
         // also orders both halves' score loads before either writes its P below)
         const float m_tile = fmaxf(m_half, exchange(m_half, ok));
@@ -595,12 +596,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
       const bool valid = grow < w.len;
       const int tok = w.tok0 + grow;
       const size_t obase = ((size_t)tok * args.num_q_heads + w.head) * args.head_dim + w.vpart * Cfg::kDv;
+      // O leaves TMEM two 32-column chunks per wait; once the last chunks are in
+      // registers the warp signals o_empty, before its stores.
+      constexpr int kOC = kHO / 32;               // 32-column chunks of this half
+      constexpr int kOG = kOC >= 2 ? 2 : 1;       // chunks per TMEM wait
 #pragma unroll 1
-      for (int c = 0; c < kHO / 32; ++c) {
-        uint32_t oh[32];
-        tmem_ld_x32(tmem + lane_off + kColO + half * kHO + c * 32, oh);
+      for (int cg = 0; cg < kOC; cg += kOG) {
+        uint32_t ohg[kOG][32];
+#pragma unroll
+        for (int k = 0; k < kOG; ++k) tmem_ld_x32(tmem + lane_off + kColO + half * kHO + (cg + k) * 32, ohg[k]);
         tmem_ld_wait();
-        const int col = half * kHO + c * 32;
+        if (cg + kOG >= kOC) {
+          // O has been read out: the next unit's first value MMA may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (!PAIR || leader) mbar_arrive(&bars->o_empty);
+            else mbar_arrive_cluster(smem_u32(&bars->o_empty) & kPeerBitMask);
+          }
+        }
+#pragma unroll
+      for (int k = 0; k < kOG; ++k) {
+        const uint32_t* oh = ohg[k];
+        const int col = half * kHO + (cg + k) * 32;
         if (valid && w.vpart * Cfg::kDv + col < args.head_dim) {
           // a row segment of 32 columns: 128 bytes (f32) or 64 bytes (bf16), written with
           // 32-byte stores where the output is 32-byte aligned (half the store
@@ -632,15 +650,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
           }
         }
       }
+      }
       if (half == 0 && valid && w.vpart == 0 && args.lse != nullptr)
         args.lse[(size_t)w.head * args.total_tokens + tok] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
-      // O has been read out: the next unit's first value MMA may overwrite it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (!PAIR || leader) mbar_arrive(&bars->o_empty);
-        else mbar_arrive_cluster(smem_u32(&bars->o_empty) & kPeerBitMask);
-      }
       g += w.ntiles;
       ++unit_iter;
     }
