@@ -17,7 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgemma_attn.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m global_interleaved_layers_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python global_interleaved_layers_b200/build.py` "
+                      "(or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -70,12 +71,14 @@ _lib.gemma_attn_decode_num_splits.argtypes = [_PP, _I, _I, _I, ctypes.POINTER(ct
 _lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_tile_plan.argtypes = [_I, _I, _P, _I, _I, _I, _P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
 _lib.gemma_attn_decode_noalloc.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]
+_lib.gemma_attn_cache_append.argtypes = [_PP, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P]
 _lib.gemma_attn_check.argtypes = [_P]
 _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
 _lib.gemma_attn_selftest_timeout.argtypes = [_P, _P]
 for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_attn_decode",
            "gemma_attn_decode_num_splits", "gemma_attn_combine", "gemma_attn_tile_plan", "gemma_attn_check",
            "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc", "gemma_attn_selftest_timeout",
+           "gemma_attn_cache_append",
            "gemma_attn_prefill_rotate", "gemma_attn_prefill_attend"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -178,6 +181,14 @@ def gemma_attn_decode_noalloc(p: GemmaAttnParams, q, new_k, new_v, k_cache, v_ca
                                           _ptr(v_cache), cache_layout, cache_capacity, _ptr(cache_seqlens), batch,
                                           n_q, max_cache_len, num_splits, _ptr(out), _ptr(lse), _stream(stream)),
            "gemma_attn_decode_noalloc")
+
+
+def gemma_attn_cache_append(p: GemmaAttnParams, new_k, new_v, k_cache, v_cache, cache_layout: int,
+                            cache_capacity: int, cache_seqlens, batch: int, n_q: int, stream=None) -> None:
+    """New tokens' K (and V) rows into the cache at slot position mod window (ring) or row position."""
+    _check(_lib.gemma_attn_cache_append(ctypes.byref(p), _ptr(new_k), _ptr(new_v), _ptr(k_cache), _ptr(v_cache),
+                                        cache_layout, cache_capacity, _ptr(cache_seqlens), batch, n_q,
+                                        _stream(stream)), "gemma_attn_cache_append")
 
 
 def gemma_attn_decode_num_splits(p: GemmaAttnParams, batch: int, n_q: int, max_cache_len: int) -> int:

@@ -354,6 +354,42 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   return GEMMA_ATTN_OK;
 }
 
+int gemma_attn_cache_append(const gemma_attn_params* params, const void* new_k, const void* new_v, void* k_cache,
+                            void* v_cache, int32_t cache_layout, int32_t cache_capacity,
+                            const int32_t* cache_seqlens, int32_t batch, int32_t n_q, void* stream_) {
+  t_launches = 0;
+  int rc = check_params(params);
+  if (rc != GEMMA_ATTN_OK) return rc;
+  const bool global = params->kind == GEMMA_ATTN_GLOBAL;
+  if (!new_k || !k_cache || !cache_seqlens) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (batch < 1 || n_q < 1 || cache_capacity < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
+  const bool keys_rotated = (cache_layout & GEMMA_ATTN_CACHE_KEYS_ROTATED) != 0;
+  if (keys_rotated && global) return GEMMA_ATTN_ERR_INVALID_ARG;  // the K=V tensor is also the values
+  cache_layout &= ~GEMMA_ATTN_CACHE_KEYS_ROTATED;
+  if (cache_layout != GEMMA_ATTN_CACHE_CONTIGUOUS && cache_layout != GEMMA_ATTN_CACHE_RING)
+    return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (cache_layout == GEMMA_ATTN_CACHE_RING && (global || cache_capacity != params->window))
+    return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (((uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
+    return GEMMA_ATTN_ERR_MISALIGNED;
+  AppendArgs a{};
+  a.new_k = static_cast<const uint16_t*>(new_k);
+  a.new_v = static_cast<const uint16_t*>(new_v);
+  a.k_cache = static_cast<uint16_t*>(k_cache);
+  a.v_cache = static_cast<uint16_t*>(v_cache);
+  a.cache_seqlens = cache_seqlens;
+  a.batch = batch; a.n_q = n_q; a.num_kv_heads = params->num_kv_heads; a.head_dim = params->head_dim;
+  a.capacity = cache_capacity;
+  a.ring = cache_layout == GEMMA_ATTN_CACHE_RING;
+  a.keys_rotated = keys_rotated ? 1 : 0;
+  a.r = rotated_pairs(params->rope_p, params->head_dim);
+  a.log2_base = log2((double)params->rope_base);
+  if (launch_cache_append(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
+  t_launches = 1;
+  return GEMMA_ATTN_OK;
+}
+
 int gemma_attn_combine(const float* partial_o, const float* partial_lse, int32_t num_splits, int32_t rows,
                        int32_t head_dim, int32_t out_dtype, void* out, float* lse, void* stream_) {
   t_launches = 0;

@@ -88,4 +88,19 @@ struct CombineArgs {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 cudaError_t launch_timeout_selftest(int* gave_up, cudaStream_t stream);
 
+// New tokens' rows into a decode cache (ring slot p mod capacity, or row p).
+struct AppendArgs {
+  const uint16_t* new_k;    // [B, n_q, Hkv, d]
+  const uint16_t* new_v;    // [B, n_q, Hkv, d] or null (K=V)
+  uint16_t* k_cache;        // [B, Hkv, capacity, d]
+  uint16_t* v_cache;        // same, or null (K=V)
+  const int32_t* cache_seqlens;
+  int batch, n_q, num_kv_heads, head_dim, capacity;
+  int ring;
+  int keys_rotated;         // store the key rotated for its position (first r pairs)
+  int r;
+  double log2_base;
+};
+cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream);
+
 }  // namespace gattn

@@ -5,4 +5,5 @@
 #include "prefill.cu"
 #include "decode.cu"
 #include "decode_noalloc.cu"
+#include "append.cu"
 #include "selftest.cu"

@@ -210,6 +210,33 @@ int gemma_attn_decode_noalloc(const gemma_attn_params* params, const void* q, co
                               int32_t max_cache_len, int32_t num_splits, void* out, float* lse,
                               void* stream);
 
+/*
+ * KV-cache append: the rows of the new tokens join the cache ("Visual guide to Gemma 4",
+ * sections "K=V technique" and "GQA": one stored KV tensor per KV head; section "p-RoPE":
+ * which pairs a stored key has rotated). Token i of sequence b, at position
+ * p = cache_seqlens[b] + i, is written to slot p mod window (GEMMA_ATTN_CACHE_RING) or to
+ * row p (GEMMA_ATTN_CACHE_CONTIGUOUS) of k_cache (and v_cache for LOCAL). With
+ * GEMMA_ATTN_CACHE_KEYS_ROTATED (LOCAL only) the key is stored rotated for p (pairs
+ * (j, j + d/2), j < r = floor(rope_p * d / 2), angle p * rope_base^(-2j/d), fp32 math from
+ * the bf16 inputs, bf16 result), the form gemma_attn_decode reads from such a cache;
+ * values and GLOBAL K=V rows are copied unchanged.
+ *   Arguments: new_k / new_v [batch, n_q, num_kv_heads, head_dim] bf16 (new_v NULL for
+ *   GLOBAL), k_cache / v_cache and cache_layout / cache_capacity as gemma_attn_decode
+ *   (v_cache NULL for GLOBAL), cache_seqlens [batch] int32 device: the tokens cached
+ *   before these (not modified: the caller advances it by n_q). All device pointers,
+ *   16-byte aligned; the caller owns every buffer.
+ *   Order: call it after the decode / verify step that read these tokens from new_k /
+ *   new_v. In a W-slot ring the new rows overwrite the slots of positions p - W, which
+ *   that step's earlier queries still see (p - W > position - W for a query before p).
+ *   Errors: GEMMA_ATTN_ERR_INVALID_ARG / _MISALIGNED as gemma_attn_decode, before any
+ *   launch. A contiguous-cache position p >= cache_capacity (or a negative length) writes
+ *   nothing for that row and records GEMMA_ATTN_ERR_SEQLEN in the device status word,
+ *   read by gemma_attn_check.
+ */
+int gemma_attn_cache_append(const gemma_attn_params* params, const void* new_k, const void* new_v,
+                            void* k_cache, void* v_cache, int32_t cache_layout, int32_t cache_capacity,
+                            const int32_t* cache_seqlens, int32_t batch, int32_t n_q, void* stream);
+
 /* A split count for gemma_attn_decode that fills the GPU for this shape. */
 int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,
                                  int32_t max_cache_len, int32_t* num_splits);

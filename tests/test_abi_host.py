@@ -111,6 +111,32 @@ def test_decode_argument_errors():
     assert e.value.status == G.ERR_UNSUPPORTED
 
 
+def test_cache_append_argument_errors():
+    p = _p(window=64)
+    fake = 1 << 20
+    pg = _p(kind=G.GLOBAL, num_q_heads=8, num_kv_heads=1, head_dim=512, rope_p=0.25)
+    cases = [
+        # ring capacity must equal the window
+        ((p, fake, fake, fake, fake, G.CACHE_RING, 32, fake, 1, 1), G.ERR_INVALID_ARG),
+        # a local layer needs its value rows, a global one has none
+        ((p, fake, None, fake, fake, G.CACHE_RING, 64, fake, 1, 1), G.ERR_INVALID_ARG),
+        ((pg, fake, fake, fake, None, G.CACHE_CONTIGUOUS, 64, fake, 1, 1), G.ERR_INVALID_ARG),
+        # no ring and no rotated keys for a global layer's K=V cache
+        ((pg, fake, None, fake, None, G.CACHE_RING, 64, fake, 1, 1), G.ERR_INVALID_ARG),
+        ((pg, fake, None, fake, None, G.CACHE_CONTIGUOUS | G.CACHE_KEYS_ROTATED, 64, fake, 1, 1), G.ERR_INVALID_ARG),
+        # empty batch, no new tokens, unknown layout bits
+        ((p, fake, fake, fake, fake, G.CACHE_RING, 64, fake, 0, 1), G.ERR_INVALID_ARG),
+        ((p, fake, fake, fake, fake, G.CACHE_RING, 64, fake, 1, 0), G.ERR_INVALID_ARG),
+        ((p, fake, fake, fake, fake, G.CACHE_RING | 0x40, 64, fake, 1, 1), G.ERR_INVALID_ARG),
+        # rows must be 16-byte aligned
+        ((p, fake + 2, fake, fake, fake, G.CACHE_RING, 64, fake, 1, 1), G.ERR_MISALIGNED),
+    ]
+    for args, code in cases:
+        with pytest.raises(G.GemmaAttnError) as e:
+            G.gemma_attn_cache_append(*args, stream=0)
+        assert e.value.status == code, args
+
+
 def test_workspace_sizes():
     # local p = 1: full rotated q and k copies; global p = 0.25, d = 512: 2 of 8 chunks
     T = 1000
