@@ -2,7 +2,9 @@
 
 A step is one pass of the hot path over the E2B-shaped prefill block: L = 8192 tokens,
 4 sliding-window layers (W = 512, 8/4 heads, d = 256) and 1 global layer (8/1 heads,
-d = 512, K=V, p-RoPE p = 0.25). `value` is unmasked prefill TFLOP/s of that block.
+d = 512, K=V, p-RoPE p = 0.25). `value` is unmasked prefill TFLOP/s of that block, its
+ten launches (rotated side copy + attention per layer) replayed as one CUDA graph; the
+same calls launched one by one are reported as per_kind.e2b_block_eager.
 In the same run the decode path (split-KV + combine) is timed on the long-context
 decode shape (batch 8, 32/4 heads, global K=V cache of 131072 tokens at d = 512;
 local 1024-slot ring at d = 256, 32/16 heads) and reported in HBM GB/s.
@@ -350,35 +352,22 @@ def main():
     total_flops = sum(l["flops"] for l in layers)
 
     stream = torch.cuda.current_stream()
-    kind_ev = {}  # per layer index: list of (start, end) events, recorded on the launch stream
-    attend_ev = {}  # the same for the attention phase alone
+    kind_ev = {}  # per layer index: the layer's time (ms) in each timed step
+    attend_ev = {}  # the same for its attention kernel alone
 
-    def run_layer(li, record=False):
-        # one layer = the prefill's two phases back to back (exactly what gemma_attn_prefill
-        # runs); the event between them times the attention kernel by itself
+    def run_layer(li):
+        # one layer = the prefill's two phases back to back (exactly what gemma_attn_prefill runs)
         l = layers[li]
         call = (l["p"], l["q"], l["k"], l["v"], l["out"], None, pos, cu, 1, L, L, ws, ws.numel(), stream)
-        if record:
-            e0 = torch.cuda.Event(enable_timing=True)
-            ea = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
         G.gemma_attn_prefill_rotate(*call)
         n = G.gemma_attn_last_launch_count()
-        if record:
-            ea.record(stream)
         G.gemma_attn_prefill_attend(*call)
-        n += G.gemma_attn_last_launch_count()
-        if record:
-            e1.record(stream)
-            kind_ev.setdefault(li, []).append((e0, e1))
-            attend_ev.setdefault(li, []).append((ea, e1))
-        return n
+        return n + G.gemma_attn_last_launch_count()
 
-    def step(record=False):
+    def step():
         n = 0
         for li in range(len(layers)):
-            n += run_layer(li, record)
+            n += run_layer(li)
         return n
 
     log("prefill warmup")
@@ -386,6 +375,26 @@ def main():
         step()
     G.gemma_attn_check()
     torch.cuda.synchronize()
+
+    # The timed step is the block's ten launches (rotate + attend per layer) recorded once
+    # as a CUDA graph and replayed (global_interleaved_layers_b200.block), as a serving
+    # loop runs a fixed-shape step. Two events inside the graph time the global layer's
+    # attention kernel (each recorded event costs the stream a few microseconds, so there
+    # are no others). The same calls launched one by one, with events around every layer,
+    # are timed after it (per_kind.e2b_block_eager and the per-layer figures).
+    from global_interleaved_layers_b200.block import BlockLayer, InterleavedBlock
+    blk = InterleavedBlock([BlockLayer(l["p"], l["q"], l["k"], l["v"], l["out"], None, pos, cu, 1, L, L, ws)
+                            for l in layers])
+    glob = [li for li, l in enumerate(layers) if l["spec"].kind == W.GLOBAL]
+    loc = [li for li, l in enumerate(layers) if l["spec"].kind == W.LOCAL]
+    att0 = torch.cuda.Event(enable_timing=True, external=True)
+    att1 = torch.cuda.Event(enable_timing=True, external=True)
+    gev = [((None, att0, att1) if li == glob[0] else None) for li in range(len(layers))]
+    launches_per_step = blk.capture(events=gev)
+    for _ in range(args.warmup):
+        blk.replay()
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
     log("prefill timed")
 
     step_events = []
@@ -398,9 +407,13 @@ def main():
             s0 = torch.cuda.Event(enable_timing=True)
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
-            launches += step(record=True)
+            blk.replay()
             s1.record(stream)
+            launches += launches_per_step
             step_events.append((s0, s1))
+            # the graph's events are re-recorded by every replay: read them now
+            s1.synchronize()
+            attend_ev.setdefault(glob[0], []).append(att0.elapsed_time(att1))
         torch.cuda.synchronize()
         barrier()
     clk = clocks.summary()
@@ -409,17 +422,48 @@ def main():
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / args.steps
     value = world * total_flops * args.steps / (total_ms * 1e-3) / 1e12
+    blk.graph = None  # release the graph before its buffers are reused below
 
-    per_layer_ms = {li: float(np.mean([a.elapsed_time(b) for a, b in evs])) for li, evs in kind_ev.items()}
-    glob = [li for li, l in enumerate(layers) if l["spec"].kind == W.GLOBAL]
-    loc = [li for li, l in enumerate(layers) if l["spec"].kind == W.LOCAL]
+    # the same step launched call by call (no graph), with events around every layer
+    eager_events = []
+    layer_events = []
+    barrier()
+    for _ in range(args.steps):
+        flush_l2()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        evs = []
+        for li in range(len(layers)):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run_layer(li)
+            e1.record(stream)
+            evs.append((e0, e1))
+        s1.record(stream)
+        eager_events.append((s0, s1))
+        layer_events.append(evs)
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    barrier()
+    eager_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in eager_events])))
+    for evs in layer_events:
+        for li, (e0, e1) in enumerate(evs):
+            kind_ev.setdefault(li, []).append(e0.elapsed_time(e1))
+    block_eager = {"ms": eager_ms, "tflops": world * total_flops / (eager_ms * 1e-3) / 1e12,
+                   "launches": launches_per_step,
+                   "note": "the timed step's calls launched one by one from Python (no CUDA graph), "
+                           "with events around every layer (per_kind.local_prefill / global_prefill)"}
+
+    per_layer_ms = {li: float(np.mean(v)) for li, v in kind_ev.items()}
     g_ms = float(np.mean([per_layer_ms[i] for i in glob]))
     l_ms = float(np.mean([per_layer_ms[i] for i in loc]))
     g_flops = layers[glob[0]]["flops"]
     l_flops = layers[loc[0]]["flops"]
     g_tflops = g_flops / (g_ms * 1e-3) / 1e12
     # the dominant kernel (the global layer's attention) per launch, timed inside the step
-    attend_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in attend_ev[glob[0]]])))
+    attend_ms = max_over_ranks(float(np.mean(attend_ev[glob[0]])))
     attend_tflops = g_flops / (attend_ms * 1e-3) / 1e12
     l_tflops = l_flops / (l_ms * 1e-3) / 1e12
     peak_t = peaks["bf16_tflops_sustained"]
@@ -507,12 +551,14 @@ def main():
             "local_prefill": {"tflops": l_tflops, "ms": l_ms, "frac_of_peak": l_tflops / peak_t,
                               "tile_geometry_ceiling": local_ceiling},
             "global_prefill": {"tflops": g_tflops, "ms": g_ms, "frac_of_peak": g_tflops / peak_t},
+            "e2b_block_eager": block_eager,
         },
         "roofline": {"bound": "tensor", "achieved": attend_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attend_tflops / peak_t, "kernel_ms": attend_ms, "traffic": ncu_traffic(),
                      "traffic_unit": "bytes per launch",
                      "kernel": "prefill_kernel<512, 1>: the global layer's attention phase, timed with "
-                               "CUDA events inside the timed step (per_kind.global_prefill also counts the "
+                               "CUDA events recorded inside the timed step's graph (per_kind.global_prefill, from "
+                               "the call-by-call run, also counts the "
                                "rotated side copy)",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -625,6 +671,31 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
             # (the kernel rotates every key) is reported beside it
             res["local_decode"] = measure(layout | G.CACHE_KEYS_ROTATED)
             res["local_decode_unrotated_cache"] = measure(layout)
+
+        # the step's new rows into the cache (after the decode that read them beside it)
+        app_layout = layout if layer.k_eq_v else (layout | G.CACHE_KEYS_ROTATED)
+        # the contiguous cache is exactly full here: time the append over its last n_q rows
+        app_lens = lens - n_q if layer.k_eq_v else lens
+        for _ in range(args.warmup):
+            G.gemma_attn_cache_append(p, nk, nv, kc, vc, app_layout, cap, app_lens, B, n_q, stream)
+        torch.cuda.synchronize()
+        app_evs = []
+        barrier()
+        for _ in range(args.steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            G.gemma_attn_cache_append(p, nk, nv, kc, vc, app_layout, cap, app_lens, B, n_q, stream)
+            e1.record(stream)
+            app_evs.append((e0, e1))
+        torch.cuda.synchronize()
+        G.gemma_attn_check()
+        barrier()
+        app_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in app_evs])))
+        app_bytes = 2 * B * n_q * Hkv * d * 2 * (1 if layer.k_eq_v else 2)  # rows read + written
+        res["global_cache_append" if layer.kind == W.GLOBAL else "local_cache_append"] = {
+            "us": app_ms * 1e3, "bytes": app_bytes, "launches": 1,
+            "note": "one launch per decode step; launch-bound (the rows are a few hundred KB)"}
         del kc, vc
         torch.cuda.empty_cache()
     return res
