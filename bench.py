@@ -577,14 +577,21 @@ def main():
 
 
 def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
-    wl = W.long_decode()
-    B, n_q = wl.batch, wl.n_q
+    res = {}
     gen = torch.Generator(device=dev)
     gen.manual_seed(99)
-    res = {}
+    # the long-context decode step, then the 4-token verify of the ragged 31B-shaped batch
+    for wl, tag in ((W.long_decode(), "decode"), (W.ragged_31b()[1], "verify")):
+        bench_decode_workload(G, torch, dev, stream, flush_l2, peaks, args, max_over_ranks, barrier, gen, wl, tag,
+                              res)
+    return res
+
+
+def bench_decode_workload(G, torch, dev, stream, flush_l2, peaks, args, max_over_ranks, barrier, gen, wl, tag, res):
+    B, n_q = wl.batch, wl.n_q
     for layer in wl.layers:
         Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
-        ctx = wl.cache_lens[0]
+        ctx = max(wl.cache_lens)
         if layer.kind == W.GLOBAL:
             cap = ctx
             layout = G.CACHE_CONTIGUOUS
@@ -600,7 +607,7 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
         q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
         nk = torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
         nv = None if layer.k_eq_v else torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
-        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        lens = torch.tensor(list(wl.cache_lens), dtype=torch.int32, device=dev)
         p = G.params(layer.kind, Hq, Hkv, d, window=layer.window, rope_p=layer.rope_p, rope_base=layer.rope_base,
                      softmax_scale=layer.softmax_scale)
         splits = G.gemma_attn_decode_num_splits(p, B, n_q, ctx)
@@ -609,7 +616,7 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
         pl = torch.empty((splits, rows), dtype=torch.float32, device=dev)
         out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
 
-        log(f"decode kind={layer.kind}")
+        log(f"{tag} kind={layer.kind}")
 
         def measure(layout):
             # one split: the one-call entry point, whose decode kernel writes the output itself;
@@ -660,17 +667,23 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
             return {"gbs": gbs, "ms": ms, "decode_kernel_ms": dec_ms, "bytes": nbytes, "splits": splits,
                     "launches": 1 if splits == 1 else 2,
                     "frac_of_hbm": gbs / peaks["hbm_gbs"],
-                    "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} ctx={ctx} " + (
+                    "shape": f"B={B} n_q={n_q} Hq={Hq} Hkv={Hkv} d={d} cache lens "
+                             f"{min(wl.cache_lens)}..{max(wl.cache_lens)} " + (
                         "K=V contiguous" if layer.k_eq_v else
                         f"ring W={layer.window}, cached keys {'stored rotated' if rotated else 'un-rotated'}")}
 
         if layer.kind == W.GLOBAL:
-            res["global_decode"] = measure(layout)
+            res[f"global_{tag}"] = measure(layout)
         else:
-            # the serving layout keeps local keys rotated in the cache; the un-rotated cache
-            # (the kernel rotates every key) is reported beside it
-            res["local_decode"] = measure(layout | G.CACHE_KEYS_ROTATED)
-            res["local_decode_unrotated_cache"] = measure(layout)
+            # the serving layout keeps local keys rotated in the cache; for the decode step
+            # the un-rotated cache (the kernel rotates every key) is reported beside it
+            res[f"local_{tag}"] = measure(layout | G.CACHE_KEYS_ROTATED)
+            if tag == "decode":
+                res["local_decode_unrotated_cache"] = measure(layout)
+        if tag != "decode":
+            del kc, vc
+            torch.cuda.empty_cache()
+            continue
 
         # the step's new rows into the cache (after the decode that read them beside it)
         app_layout = layout if layer.k_eq_v else (layout | G.CACHE_KEYS_ROTATED)
@@ -698,7 +711,6 @@ def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
             "note": "one launch per decode step; launch-bound (the rows are a few hundred KB)"}
         del kc, vc
         torch.cuda.empty_cache()
-    return res
 
 
 def run_case(args):
