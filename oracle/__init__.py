@@ -12,7 +12,9 @@ pages are silent.
 Pinned by ``tests/test_oracle_pins.py`` (closed forms for the rotation sign, pair
 layout, frequencies and the p cut-off; window and causal special cases; GQA
 replication; shift invariance; an independent SDPA special case; split/combine
-equivalence; brute-force tile counts).
+equivalence; brute-force tile counts), and the bidirectional 2D-RoPE routine by
+``tests/test_oracle_pins_2d.py`` (each half a 1D rotation, shift invariance, SDPA
+without a mask, patch permutation, GQA, the all-full tile plan).
 """
 from __future__ import annotations
 
@@ -30,6 +32,7 @@ _lib = None
 
 LOCAL = 0
 GLOBAL = 1
+BIDIR = 2  # bidirectional attention over an image's patches, 2D RoPE
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +61,11 @@ def _load():
         lib.oracle_tile_plan.restype = ctypes.c_longlong
         lib.oracle_rope.argtypes = [P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_double]
         lib.oracle_rope.restype = None
+        lib.oracle_rope2d.argtypes = [P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_double]
+        lib.oracle_rope2d.restype = None
+        lib.oracle_attention_2d.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P, P]
+        lib.oracle_attention_2d.restype = ctypes.c_int
         lib.oracle_rotated_pairs.argtypes = [ctypes.c_double, ctypes.c_int]
         lib.oracle_rotated_pairs.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
@@ -113,6 +121,40 @@ def attention(kind: int, window: int, rope_p: float, rope_base: float, scale: fl
                               cu.shape[0] - 1, _ptr(rr), n, int(klo), int(khi), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_attention rejected its arguments")
+    return out, lse
+
+
+def rope2d(x: np.ndarray, rope_base: float, pos_h: float, pos_w: float) -> np.ndarray:
+    """2D rotation of one vector (float64, length divisible by 4): first half for w, second for h."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    _load().oracle_rope2d(_ptr(x), _ptr(y), x.shape[0], float(rope_base), float(pos_h), float(pos_w))
+    return y
+
+
+def attention_2d(rope_base: float, scale: float, q: np.ndarray, k: np.ndarray, v: Optional[np.ndarray],
+                 positions_hw: np.ndarray, cu_seqlens: np.ndarray, rows: Optional[np.ndarray] = None):
+    """Bidirectional attention with 2D RoPE in fp64 (every key of the query's sequence).
+
+    q [T, Hq, d], k / v [T, Hkv, d] bf16 bits (v None: K=V); positions_hw [T, 2] int (h, w).
+    Returns (out [R, Hq, d], lse [R, Hq]) float64 for R = len(rows) (or T).
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = None if v is None else np.ascontiguousarray(v, dtype=np.uint16)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    hw = np.ascontiguousarray(positions_hw, dtype=np.int32).reshape(T, 2)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n = T if rr is None else rr.shape[0]
+    out = np.zeros((n, Hq, d), dtype=np.float64)
+    lse = np.zeros((n, Hq), dtype=np.float64)
+    rc = lib.oracle_attention_2d(float(rope_base), float(scale), Hq, Hkv, d, _ptr(q), _ptr(k), _ptr(v), _ptr(hw),
+                                 _ptr(cu), cu.shape[0] - 1, _ptr(rr), n, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attention_2d rejected its arguments")
     return out, lse
 
 

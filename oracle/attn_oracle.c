@@ -17,6 +17,10 @@
  *       section "K=V technique".
  *   - p-RoPE (only the top p fraction of rotary pairs rotated, the
  *       low-frequency remainder passed through): guide, section "p-RoPE".
+ *   - 2D RoPE of the vision encoder's patches (the embedding split in two
+ *       parts, one encoding the horizontal position w, the other the vertical
+ *       position h): guide, section "Vision encoder"; the encoder's attention
+ *       over an image's patches is bidirectional (a ViT sees every patch).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   window = keys with  pos_q - W < pos_k <= pos_q  (W keys including self);
@@ -26,6 +30,9 @@
  *   theta_j = base^(-2j/d), counter-clockwise rotation by pos * theta_j,
  *   applied to q and to the key copy used for scores; values are the
  *   un-rotated tensor (for K=V this is the single stored tensor).
+ *   2D RoPE: dims [0, d/2) rotated for w and dims [d/2, d) for h, each half
+ *   by the 1D rule above with d/2 in place of d (pairs (j, j + d/4),
+ *   theta_j = base^(-2j/(d/2))); bidirectional = every key of the sequence.
  *
  * Every computation widens the bf16 inputs exactly to double and works in
  * double; angles, cosines and sines are double.
@@ -40,6 +47,7 @@
 
 #define ORACLE_LOCAL 0
 #define ORACLE_GLOBAL 1
+#define ORACLE_BIDIR 2
 
 static double bf16_to_double(uint16_t bits) {
   uint32_t u = ((uint32_t)bits) << 16;
@@ -83,6 +91,19 @@ void oracle_rope(const double* x, double* y, int d, double rope_p, double rope_b
   free(cs);
 }
 
+/* 2D rotation of x (length d, d divisible by 4): the first half of the dims for the
+ * horizontal position w, the second half for the vertical position h, each half by the
+ * 1D rotation of a d/2-dim vector (every pair rotated). */
+void oracle_rope2d(const double* x, double* y, int d, double rope_base, double pos_h, double pos_w) {
+  const int half = d / 2, pairs = d / 4;
+  double* cs = (double*)malloc(sizeof(double) * 2 * (pairs > 0 ? pairs : 1));
+  for (int j = 0; j < pairs; ++j) rope_angle(pos_w, j, half, rope_base, &cs[2 * j], &cs[2 * j + 1]);
+  rope_apply(x, y, half, pairs, cs);
+  for (int j = 0; j < pairs; ++j) rope_angle(pos_h, j, half, rope_base, &cs[2 * j], &cs[2 * j + 1]);
+  rope_apply(x + half, y + half, half, pairs, cs);
+  free(cs);
+}
+
 static int seq_of_token(const int32_t* cu_seqlens, int num_seqs, int t) {
   int lo = 0, hi = num_seqs - 1;
   while (lo < hi) {
@@ -93,6 +114,7 @@ static int seq_of_token(const int32_t* cu_seqlens, int num_seqs, int t) {
 }
 
 static int key_visible(int kind, int window, int32_t pos_q, int32_t pos_k) {
+  if (kind == ORACLE_BIDIR) return 1;  /* every key of the sequence */
   if (pos_k > pos_q) return 0;
   if (kind == ORACLE_LOCAL && !(pos_q - window < pos_k)) return 0;
   return 1;
@@ -195,6 +217,69 @@ int oracle_attention(int kind, int window, double rope_p, double rope_base, doub
     free(qv); free(qr); free(kv); free(kr); free(acc); free(z);
   }
   free(table);
+  return 0;
+}
+
+/*
+ * Bidirectional attention with 2D RoPE (the vision encoder's patches).
+ *   q [T, Hq, d], k [T, Hkv, d], v [T, Hkv, d] as bf16 bits; v == NULL means K=V.
+ *   positions_hw [T, 2]: (h, w) of each token; cu_seqlens [num_seqs + 1]: each image's
+ *   patches, which see every patch of their own image and nothing else.
+ *   rows / n_rows, out [n_rows, Hq, d], lse [n_rows, Hq] (may be NULL) as in
+ *   oracle_attention. Scores use the rotated q and k, values the un-rotated tensor.
+ */
+int oracle_attention_2d(double rope_base, double scale, int Hq, int Hkv, int d,
+                        const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const int32_t* positions_hw, const int32_t* cu_seqlens, int num_seqs,
+                        const int32_t* rows, int n_rows, double* out, double* lse) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || d % 4 != 0 || num_seqs <= 0) return -1;
+  const int group = Hq / Hkv;
+  const uint16_t* vv = v ? v : k;
+  int T = cu_seqlens[num_seqs];
+  if (!rows) n_rows = T;
+  long long jobs = (long long)n_rows * Hq;
+#pragma omp parallel
+  {
+    double* qv = (double*)malloc(sizeof(double) * d);
+    double* qr = (double*)malloc(sizeof(double) * d);
+    double* kv = (double*)malloc(sizeof(double) * d);
+    double* kr = (double*)malloc(sizeof(double) * d);
+    double* acc = (double*)malloc(sizeof(double) * d);
+    int cap = 0;
+    double* z = NULL;
+#pragma omp for schedule(dynamic, 4)
+    for (long long job = 0; job < jobs; ++job) {
+      int ri = (int)(job / Hq), h = (int)(job % Hq);
+      int t = rows ? rows[ri] : ri;
+      int s = seq_of_token(cu_seqlens, num_seqs, t);
+      int beg = cu_seqlens[s], end = cu_seqlens[s + 1];
+      int g = h / group;
+      if (end - beg > cap) { cap = end - beg; z = (double*)realloc(z, sizeof(double) * cap); }
+      for (int i = 0; i < d; ++i) qv[i] = bf16_to_double(q[((size_t)t * Hq + h) * d + i]);
+      oracle_rope2d(qv, qr, d, rope_base, positions_hw[2 * t], positions_hw[2 * t + 1]);
+      double zmax = -INFINITY;
+      for (int u = beg; u < end; ++u) {
+        for (int i = 0; i < d; ++i) kv[i] = bf16_to_double(k[((size_t)u * Hkv + g) * d + i]);
+        oracle_rope2d(kv, kr, d, rope_base, positions_hw[2 * u], positions_hw[2 * u + 1]);
+        double dot = 0.0;
+        for (int i = 0; i < d; ++i) dot += qr[i] * kr[i];
+        z[u - beg] = scale * dot;
+        if (z[u - beg] > zmax) zmax = z[u - beg];
+      }
+      double* o = out + ((size_t)ri * Hq + h) * d;
+      double denom = 0.0;
+      for (int i = 0; i < d; ++i) acc[i] = 0.0;
+      for (int u = beg; u < end; ++u) {
+        double w = exp(z[u - beg] - zmax);
+        denom += w;
+        const uint16_t* vrow = vv + ((size_t)u * Hkv + g) * d;
+        for (int i = 0; i < d; ++i) acc[i] += w * bf16_to_double(vrow[i]);
+      }
+      for (int i = 0; i < d; ++i) o[i] = acc[i] / denom;
+      if (lse) lse[(size_t)ri * Hq + h] = zmax + log(denom);
+    }
+    free(qv); free(qr); free(kv); free(kr); free(acc); free(z);
+  }
   return 0;
 }
 
