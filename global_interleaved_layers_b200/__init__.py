@@ -24,6 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 LOCAL = 0
 GLOBAL = 1
+BIDIR = 2  # vision patches: bidirectional, 2D RoPE; positions are [T, 2] (h, w); prefill only
 CACHE_CONTIGUOUS = 0
 CACHE_RING = 1
 CACHE_KEYS_ROTATED = 0x100  # OR-ed into the layout (local layers): cached keys stored rotated

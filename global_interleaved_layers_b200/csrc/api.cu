@@ -65,11 +65,15 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int check_params(const gemma_attn_params* p) {
   if (!p) return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (p->kind != GEMMA_ATTN_LOCAL && p->kind != GEMMA_ATTN_GLOBAL) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (p->kind != GEMMA_ATTN_LOCAL && p->kind != GEMMA_ATTN_GLOBAL && p->kind != GEMMA_ATTN_BIDIR)
+    return GEMMA_ATTN_ERR_INVALID_ARG;
   if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0)
     return GEMMA_ATTN_ERR_INVALID_ARG;
   const int d = p->head_dim;
   if (d != 32 && d != 64 && d != 128 && d != 256 && d != 512) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  // the 2D rotation turns every pair of both halves: p = 1, whole 64-dim chunks
+  if (p->kind == GEMMA_ATTN_BIDIR && p->rope_p != 1.f) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (p->kind == GEMMA_ATTN_BIDIR && d < 64) return GEMMA_ATTN_ERR_UNSUPPORTED;
   if (p->kind == GEMMA_ATTN_LOCAL && p->window < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (!(p->rope_p >= 0.f && p->rope_p <= 1.f)) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (!(p->rope_base > 0.f) || !(p->softmax_scale > 0.f)) return GEMMA_ATTN_ERR_INVALID_ARG;
@@ -162,6 +166,7 @@ int prefill_phases(const gemma_attn_params* params, const void* q, const void* k
   int rc = check_params(params);
   if (rc != GEMMA_ATTN_OK) return rc;
   const bool global = params->kind == GEMMA_ATTN_GLOBAL;
+  const bool bidir = params->kind == GEMMA_ATTN_BIDIR;
   if (!q || !k || !out || !positions || !cu_seqlens) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (global != (v == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (num_seqs < 1 || total_tokens < 1 || max_seqlen < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
@@ -180,7 +185,15 @@ int prefill_phases(const gemma_attn_params* params, const void* q, const void* k
   uint16_t* vpad = reinterpret_cast<uint16_t*>(ws + L.v_off);
   const double log2_base = log2((double)params->rope_base);
 
-  if (L.mask && (phases & kPhaseRotate)) {
+  if (bidir && (phases & kPhaseRotate)) {
+    // whole rows rotated (positions are (h, w) pairs), queries and keys in one launch
+    Rope2dArgs ra;
+    ra.src = static_cast<const uint16_t*>(q); ra.dst = qside; ra.heads = Hq;
+    ra.src2 = static_cast<const uint16_t*>(k); ra.dst2 = kside; ra.heads2 = Hkv;
+    ra.positions_hw = positions; ra.tokens = total_tokens; ra.d = d; ra.log2_base = log2_base;
+    if (launch_rope2d_side(ra, stream) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
+    ++t_launches;
+  } else if (L.mask && (phases & kPhaseRotate)) {
     RopeArgs ra;
     ra.positions = positions; ra.tokens = total_tokens; ra.d = d; ra.r = L.r; ra.chunk_mask = L.mask;
     ra.n_out = L.n_out; ra.log2_base = log2_base;
@@ -235,8 +248,10 @@ int prefill_phases(const gemma_attn_params* params, const void* q, const void* k
   PrefillArgs a;
   a.cu_seqlens = cu_seqlens; a.out = out; a.lse = lse; a.num_seqs = num_seqs;
   a.max_qtiles = (max_seqlen + 127) / 128; a.max_seqlen = max_seqlen; a.total_tokens = total_tokens;
-  a.num_q_heads = Hq; a.group = Hq / Hkv; a.head_dim = d; a.is_local = global ? 0 : 1;
-  a.window = global ? 0 : params->window; a.softmax_scale = params->softmax_scale; a.rot_mask = L.mask;
+  a.num_q_heads = Hq; a.group = Hq / Hkv; a.head_dim = d;
+  a.is_local = params->kind == GEMMA_ATTN_LOCAL ? 1 : 0;
+  a.bidir = bidir ? 1 : 0;
+  a.window = a.is_local ? params->window : 0; a.softmax_scale = params->softmax_scale; a.rot_mask = L.mask;
   a.out_f32 = params->out_dtype == GEMMA_ATTN_OUT_F32;
   a.pair_allowed = pair_kernel_enabled();
   // 32-byte stores need the base and the row stride (head_dim elements) 32-byte aligned
@@ -286,6 +301,7 @@ int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch,
                                  int32_t max_cache_len, int32_t* num_splits) {
   int rc = check_params(params);
   if (rc != GEMMA_ATTN_OK) return rc;
+  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
   if (batch < 1 || n_q < 1 || max_cache_len < 0 || !num_splits) return GEMMA_ATTN_ERR_INVALID_ARG;
   int keys = params->kind == GEMMA_ATTN_LOCAL ? std::min(max_cache_len, params->window) : max_cache_len;
   keys += n_q;
@@ -315,6 +331,7 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   t_launches = 0;
   int rc = check_params(params);
   if (rc != GEMMA_ATTN_OK) return rc;
+  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
   const bool global = params->kind == GEMMA_ATTN_GLOBAL;
   if (!q || !new_k || !k_cache || !cache_seqlens || !partial_o || !partial_lse) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
@@ -360,6 +377,7 @@ int gemma_attn_cache_append(const gemma_attn_params* params, const void* new_k, 
   t_launches = 0;
   int rc = check_params(params);
   if (rc != GEMMA_ATTN_OK) return rc;
+  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
   const bool global = params->kind == GEMMA_ATTN_GLOBAL;
   if (!new_k || !k_cache || !cache_seqlens) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
@@ -408,9 +426,11 @@ int gemma_attn_combine(const float* partial_o, const float* partial_lse, int32_t
 int gemma_attn_tile_plan(int32_t kind, int32_t window, const int32_t* cu_seqlens_host, int32_t num_seqs,
                          int32_t bm, int32_t bn, int32_t* out, int64_t cap, int64_t* count) {
   if (!cu_seqlens_host || num_seqs < 1 || bm < 1 || bn < 1 || !count) return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (kind != GEMMA_ATTN_LOCAL && kind != GEMMA_ATTN_GLOBAL) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (kind != GEMMA_ATTN_LOCAL && kind != GEMMA_ATTN_GLOBAL && kind != GEMMA_ATTN_BIDIR)
+    return GEMMA_ATTN_ERR_INVALID_ARG;
   if (kind == GEMMA_ATTN_LOCAL && window < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
   const int is_local = kind == GEMMA_ATTN_LOCAL;
+  const int bidir = kind == GEMMA_ATTN_BIDIR;
   int64_t n = 0;
   for (int s = 0; s < num_seqs; ++s) {
     const int len = cu_seqlens_host[s + 1] - cu_seqlens_host[s];
@@ -418,13 +438,13 @@ int gemma_attn_tile_plan(int32_t kind, int32_t window, const int32_t* cu_seqlens
     const int nqt = (len + bm - 1) / bm;
     for (int qt = 0; qt < nqt; ++qt) {
       int lo, hi;
-      kv_tile_range(is_local, window, len, qt, bm, bn, &lo, &hi);
+      kv_tile_range(is_local, window, len, qt, bm, bn, &lo, &hi, bidir);
       for (int kt = lo; kt < hi; ++kt) {
         if (out && n < cap) {
           out[4 * n + 0] = s;
           out[4 * n + 1] = qt;
           out[4 * n + 2] = kt;
-          out[4 * n + 3] = kv_tile_class(is_local, window, len, qt, kt, bm, bn);
+          out[4 * n + 3] = kv_tile_class(is_local, window, len, qt, kt, bm, bn, bidir);
         }
         ++n;
       }

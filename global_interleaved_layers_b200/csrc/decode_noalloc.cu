@@ -66,6 +66,7 @@ extern "C" int gemma_attn_decode_noalloc(const gemma_attn_params* params, const 
                                          void* stream_) {
   using namespace gattn;
   if (!params) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
   if (params->kind != GEMMA_ATTN_LOCAL && params->kind != GEMMA_ATTN_GLOBAL) return GEMMA_ATTN_ERR_INVALID_ARG;
   if (params->num_q_heads <= 0 || params->num_kv_heads <= 0 || params->num_q_heads % params->num_kv_heads)
     return GEMMA_ATTN_ERR_INVALID_ARG;

@@ -19,6 +19,7 @@ struct PrefillArgs {
   int group;          // query heads per KV head
   int head_dim;       // real head dim (row stride of out); the kernel dim may be padded to 64
   int is_local;
+  int bidir;          // bidirectional (every key of the sequence); is_local is then 0
   int window;
   float softmax_scale;
   int out_f32;        // 1: write fp32 output, 0: bf16
@@ -53,6 +54,20 @@ struct RopeArgs {
   double log2_base;
 };
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream);
+
+// Rotated copies of whole rows for the 2D rotation: dims [0, d/2) rotated for w and
+// [d/2, d) for h (each half: pairs (j, j + d/4), theta_j = base^(-2j/(d/2))).
+struct Rope2dArgs {
+  const uint16_t* src;       // [T, H, d] bf16
+  uint16_t* dst;             // [T, H, d] bf16
+  const uint16_t* src2;      // optional second tensor [T, H2, d] (the keys)
+  uint16_t* dst2;
+  int heads, heads2;
+  const int32_t* positions_hw;  // [T, 2]: (h, w)
+  int tokens, d;
+  double log2_base;
+};
+cudaError_t launch_rope2d_side(const Rope2dArgs& a, cudaStream_t stream);
 
 struct DecodeArgs {
   const uint16_t* q;        // [B, n_q, Hq, d]

@@ -177,7 +177,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
     w.row0 = w.qt * kBM;
     w.kvh = w.head / args.group;
     int hi;
-    kv_tile_range(is_local, args.window, w.len, w.qt, kBM, kBN, &w.kt_lo, &hi);
+    kv_tile_range(is_local, args.window, w.len, w.qt, kBM, kBN, &w.kt_lo, &hi, args.bidir);
     w.ntiles = hi - w.kt_lo;
     return true;
   };
@@ -495,17 +495,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant_
         // A key tile that runs past the end of the sequence holds the next sequence's
         // tokens (or padding) and is masked even when its in-sequence pairs are all visible.
         const bool partial = (kt + 1) * kBN > w.len ||
-                             kv_tile_class(is_local, args.window, w.len, w.qt, kt, kBM, kBN) != kTileFull;
+                             kv_tile_class(is_local, args.window, w.len, w.qt, kt, kBM, kBN, args.bidir) != kTileFull;
         // Scores stay unscaled: the scale is folded into the exponent's FFMA (scale > 0, so
         // the max commutes with it). In a masked tile the keys a row sees are one run of
         // the half's columns, [c_lo, c_hi] (causal: key <= row; local: key > row - window;
-        // past the row's sequence end nothing, since row < len); the rest become -inf.
+        // past the row's sequence end nothing, since row < len; bidirectional: every key
+        // before the sequence end); the rest become -inf.
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
         if (partial) {
           const int k0 = kt * kBN + half * kHC;
-          const int c_hi = grow - k0;
+          const int c_hi = (args.bidir ? w.len - 1 : grow) - k0;
           const int c_lo = is_local ? grow - args.window + 1 - k0 : 0;
 #pragma unroll
           for (int c = 0; c < kHC; ++c) {

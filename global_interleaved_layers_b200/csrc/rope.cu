@@ -99,6 +99,54 @@ __global__ void rope_side_kernel(RopeArgs a) {
   if (a.heads2 > 0) rope_heads(a.src2, a.dst2, a.heads2, tok, a.d, a.n_out, j0, col0, col1, pad, c, s);
 }
 
+// 2D rotation for the vision encoder's patches ("Visual guide to Gemma 4", section
+// "Vision encoder": the embedding split in two parts that encode the horizontal and the
+// vertical position separately): dims [0, d/2) rotated by w, dims [d/2, d) by h, each
+// half as a d/2-dim rotation with pairs (j, j + d/4) and theta_j = base^(-2j/(d/2)).
+// One thread per (token, half, group of 8 pairs of that half): it computes the 8 angles
+// once and rotates those pairs in every head of the queries and the keys; every dim of
+// a row is rotated, so the copy holds whole rows.
+__global__ void rope2d_side_kernel(Rope2dArgs a) {
+  const int quarter = a.d / 4;               // pairs per half
+  const int groups = a.d / 32;               // groups of 8 pairs per half
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.tokens * 2 * groups) return;
+  const int tok = (int)(idx / (2 * groups));
+  const int part = (int)((idx / groups) % 2);  // 0: first half, position w; 1: second half, position h
+  const int j0 = (int)(idx % groups) * 8;
+  const int pos = a.positions_hw[2 * tok + (part == 0 ? 1 : 0)];
+  float c[8], s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) rope_cos_sin((double)pos, rope_inv_freq_turns(j0 + e, a.d / 2, a.log2_base), &c[e], &s[e]);
+  const int col0 = part * (a.d / 2) + j0, col1 = col0 + quarter;
+  for (int t = 0; t < 2; ++t) {
+    const uint16_t* src = t == 0 ? a.src : a.src2;
+    uint16_t* dst = t == 0 ? a.dst : a.dst2;
+    const int heads = t == 0 ? a.heads : a.heads2;
+    for (int h = 0; h < heads; ++h) {
+      const size_t row = ((size_t)tok * heads + h) * a.d;
+      float x0[8], x1[8], y0[8], y1[8];
+      unpack8(*reinterpret_cast<const uint4*>(src + row + col0), x0);
+      unpack8(*reinterpret_cast<const uint4*>(src + row + col1), x1);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        y0[e] = x0[e] * c[e] - x1[e] * s[e];
+        y1[e] = x0[e] * s[e] + x1[e] * c[e];
+      }
+      *reinterpret_cast<uint4*>(dst + row + col0) = pack8(y0);
+      *reinterpret_cast<uint4*>(dst + row + col1) = pack8(y1);
+    }
+  }
+}
+
+cudaError_t launch_rope2d_side(const Rope2dArgs& a, cudaStream_t stream) {
+  const long long total = (long long)a.tokens * 2 * (a.d / 32);
+  if (total == 0) return cudaSuccess;
+  const int threads = 128;
+  rope2d_side_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rope_side(const RopeArgs& a, cudaStream_t stream) {
   const long long total = (long long)a.tokens * a.groups_active;
   if (total == 0 || a.n_out == 0) return cudaSuccess;

@@ -48,7 +48,14 @@ extern "C" {
 
 enum {
   GEMMA_ATTN_LOCAL = 0,
-  GEMMA_ATTN_GLOBAL = 1
+  GEMMA_ATTN_GLOBAL = 1,
+  /* The vision encoder's attention over an image's patches ("Visual guide to Gemma 4",
+   * section "Vision encoder"): bidirectional (every patch of the sequence visible),
+   * 2D RoPE (dims [0, d/2) rotated for the horizontal position w, dims [d/2, d) for the
+   * vertical position h, each half as a d/2-dim rotation: pairs (j, j + d/4),
+   * theta_j = rope_base^(-2j/(d/2))). Prefill only; rope_p must be 1, head_dim >= 64,
+   * v given (separate values), window ignored. */
+  GEMMA_ATTN_BIDIR = 2
 };
 
 enum {
@@ -104,16 +111,19 @@ int gemma_attn_prefill_workspace_size(const gemma_attn_params* params, int32_t t
 /*
  * Prefill: attention of every token of a ragged batch against the earlier tokens
  * of its own sequence (flash-style; fully masked key tiles are never visited, so a
- * LOCAL layer costs O(tokens * window)).
+ * LOCAL layer costs O(tokens * window)); for GEMMA_ATTN_BIDIR against every token of
+ * its own sequence (an image's patches).
  *   q         [total_tokens, num_q_heads, head_dim] bf16, device.
  *   k         [total_tokens, num_kv_heads, head_dim] bf16, device (GLOBAL: the K=V tensor).
  *   v         same shape as k for LOCAL; must be NULL for GLOBAL (values = k, un-rotated).
  *   out       [total_tokens, num_q_heads, head_dim] bf16 or f32 (params->out_dtype), device, written.
  *   lse       [num_q_heads, total_tokens] float32 natural-log sum-exp of the scaled
  *             scores, device, written; may be NULL.
- *   positions [total_tokens] int32, device: rotary position of each token. Within a
+  *   positions [total_tokens] int32, device: rotary position of each token. Within a
  *             sequence the positions must be consecutive (p, p+1, ...): the masks are
  *             evaluated on in-sequence offsets, which equals the position rule then.
+ *             GEMMA_ATTN_BIDIR: [total_tokens, 2] int32, the (h, w) patch coordinates of
+ *             each token, in any order (no mask depends on them).
  *   cu_seqlens [num_seqs + 1] int32, device: sequence s is tokens cu[s] .. cu[s+1]-1.
  *             Lengths must be >= 1 and <= max_seqlen (violations are reported through
  *             gemma_attn_check as GEMMA_ATTN_ERR_SEQLEN).

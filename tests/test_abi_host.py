@@ -137,6 +137,37 @@ def test_cache_append_argument_errors():
         assert e.value.status == code, args
 
 
+def test_bidir_argument_rules():
+    fake = 1 << 20
+    # the 2D rotation turns every pair: rope_p must be 1
+    p = _p(kind=G.BIDIR, num_q_heads=4, num_kv_heads=4, head_dim=64, rope_p=0.5)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_prefill_workspace_size(p, 100)
+    assert e.value.status == G.ERR_INVALID_ARG
+    # whole 64-dim chunks
+    p = _p(kind=G.BIDIR, num_q_heads=4, num_kv_heads=4, head_dim=32, rope_p=1.0)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_prefill_workspace_size(p, 100)
+    assert e.value.status == G.ERR_UNSUPPORTED
+    # no decode for the vision kind
+    p = _p(kind=G.BIDIR, num_q_heads=4, num_kv_heads=4, head_dim=64, rope_p=1.0)
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_decode(p, fake, fake, fake, fake, fake, G.CACHE_CONTIGUOUS, 64, fake, 1, 1, 10, fake, fake, 1, 0)
+    assert e.value.status == G.ERR_UNSUPPORTED
+    with pytest.raises(G.GemmaAttnError) as e:
+        G.gemma_attn_decode_num_splits(p, 1, 1, 10)
+    assert e.value.status == G.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("lens", [(200, 64, 129), (1,), (128, 256)])
+def test_bidir_tile_plan_matches_oracle(lens):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    pos = np.concatenate([np.arange(n) for n in lens]).astype(np.int32)
+    got = G.gemma_attn_tile_plan(G.BIDIR, 0, cu, 128, 128)
+    want = oracle.tile_plan(oracle.BIDIR, 0, pos, cu, 128, 128)
+    np.testing.assert_array_equal(np.asarray(got).reshape(-1, 4), np.asarray(want).reshape(-1, 4))
+
+
 def test_workspace_sizes():
     # local p = 1: full rotated q and k copies; global p = 0.25, d = 512: 2 of 8 chunks
     T = 1000

@@ -26,6 +26,7 @@ import numpy as np
 
 LOCAL = 0
 GLOBAL = 1
+BIDIR = 2  # the vision encoder's bidirectional 2D-RoPE attention over an image's patches
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
