@@ -537,6 +537,7 @@ def main():
     decode = None
     if not args.no_decode:
         decode = bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier)
+    vision = bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier)
 
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -568,6 +569,7 @@ def main():
     }
     if decode is not None:
         result["per_kind"].update(decode)
+    result["per_kind"]["vision_bidir_prefill"] = vision
     if rank == 0 and not args.no_cpu_baseline:
         log("cpu baseline")
         result["cpu_baseline"] = cpu_baseline(wl)
@@ -711,6 +713,56 @@ def bench_decode_workload(G, torch, dev, stream, flush_l2, peaks, args, max_over
             "note": "one launch per decode step; launch-bound (the rows are a few hundred KB)"}
         del kc, vc
         torch.cuda.empty_cache()
+
+
+def bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
+    """The vision encoder's attention: bidirectional, 2D RoPE, 4 images of 2520 patches."""
+    wl = W.vision_batch()
+    layer = wl.layers[0]
+    T = wl.total_tokens
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    q = torch.randn((T, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    k = torch.randn((T, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn((T, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    # patches of each image row by row, 56 wide (45 x 56 = 2520)
+    idx = np.concatenate([np.arange(n) for n in wl.seq_lens])
+    hw = torch.from_numpy(np.stack([idx // 56, idx % 56], axis=1).astype(np.int32)).to(dev)
+    cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
+    p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, rope_p=1.0,
+                 rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
+    ws_bytes = G.gemma_attn_prefill_workspace_size(p, T)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    maxlen = max(wl.seq_lens)
+
+    def one():
+        G.gemma_attn_prefill(p, q, k, v, out, None, hw, cu, len(wl.seq_lens), T, maxlen, ws, ws_bytes, stream)
+
+    log("vision prefill")
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    evs = []
+    barrier()
+    for _ in range(args.steps):
+        flush_l2()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    barrier()
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+    flops = W.prefill_flops(wl.seq_lens, layer)
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"tflops": tflops, "ms": ms, "frac_of_peak": tflops / peaks["bf16_tflops_sustained"],
+            "launches": 2, "shape": f"{len(wl.seq_lens)} images x {maxlen} patches, {layer.num_q_heads} heads, "
+                                    f"d={layer.head_dim}, bidirectional, 2D RoPE (rotated copy + attention)"}
 
 
 def run_case(args):

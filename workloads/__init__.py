@@ -162,10 +162,21 @@ def ragged_31b(seed: int = 7):
     return pre, ver
 
 
+def vision_batch() -> PrefillWorkload:
+    """4 images of 2520 patches (the pages' largest patch count: 9 x 280 at a soft-token
+    budget of 280), bidirectional 2D-RoPE attention with 12 heads of 64 dims (a ViT-B-sized
+    encoder; the pages give the encoder's parameter count, not its attention shape)."""
+    layer = LayerSpec(BIDIR, 12, 12, 64, rope_p=1.0, rope_base=1e4)
+    return PrefillWorkload(name="vision_4x2520", seq_lens=(2520,) * 4, seed=0, layers=(layer,))
+
+
 def unmasked_pairs(seq_lens: Sequence[int], kind: int, window: int) -> int:
     """Number of visible (query, key) pairs for prefill with consecutive positions."""
     total = 0
     for n in seq_lens:
+        if kind == BIDIR:  # every patch sees every patch of its image
+            total += n * n
+            continue
         if kind == GLOBAL or window >= n:
             total += n * (n + 1) // 2
         else:
