@@ -38,7 +38,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of prefill_kernel<512> on the E2B global layer, from the
 # ncu capture summarised in profiles/prefill_kernel_d512_e2b_global.md. Reported only while the
 # kernel's sources still hash to the captured state; any change makes it null until re-captured.
-NCU_TRAFFIC = {"bytes": 108718336, "sources_sha256_16": "d7983e35deecf684",
+NCU_TRAFFIC = {"bytes": 109307136, "sources_sha256_16": "e2ddccf9cd60228a",
                "sources": ["global_interleaved_layers_b200/csrc/prefill.cu",
                            "global_interleaved_layers_b200/csrc/common.cuh",
                            "global_interleaved_layers_b200/csrc/tile_plan.h",
