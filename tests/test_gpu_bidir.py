@@ -65,3 +65,24 @@ def test_bidir_patch_order_and_coordinates_are_free():
     out, _ = run_prefill(G, layer, q, k, v, hw, cu, out_f32=True)
     ref, _ = oracle.attention_2d(1e4, 1 / math.sqrt(d), q, k, v, hw, cu)
     assert_close(out.cpu().numpy(), ref, "bidir shuffled")
+
+
+def test_bidir_at_the_benchmark_shape_sampled_rows():
+    """4 images x 2520 patches, 12 heads of 64 dims (the measured vision batch): sampled
+    rows of every image against the oracle."""
+    wl = W.vision_batch()
+    layer = wl.layers[0]
+    T = wl.total_tokens
+    cu = wl.cu_seqlens()
+    idx = np.concatenate([np.arange(n) for n in wl.seq_lens])
+    hw = np.stack([idx // 56, idx % 56], axis=1).astype(np.int32)
+    q = W.normal_bf16(62, 0, (T, layer.num_q_heads, layer.head_dim))
+    k = W.normal_bf16(62, 1, (T, layer.num_kv_heads, layer.head_dim))
+    v = W.normal_bf16(62, 2, (T, layer.num_kv_heads, layer.head_dim))
+    out, lse = run_prefill(G, layer, q, k, v, hw, cu, out_f32=True)
+    rng = np.random.default_rng(3)
+    rows = np.sort(np.concatenate([cu[s] + np.concatenate([[0, n - 1], rng.integers(0, n, 14)])
+                                   for s, n in enumerate(wl.seq_lens)])).astype(np.int32)
+    ref, ref_lse = oracle.attention_2d(layer.rope_base, layer.softmax_scale, q, k, v, hw, cu, rows=rows)
+    assert_close(out.cpu().numpy()[rows], ref, "vision batch, sampled rows")
+    np.testing.assert_allclose(lse.cpu().numpy().T[rows], ref_lse, atol=1e-2, rtol=0)
