@@ -1,20 +1,25 @@
-// prefill.cu -- flash-style causal attention for Gemma-4-style local (sliding
-// window) and global (K=V, p-RoPE) layers on sm_100a.
+// prefill.cu -- flash-style attention for Gemma-4-style local (sliding window, causal)
+// and global (causal, K=V, p-RoPE) layers, and the vision encoder's bidirectional
+// layers, on sm_100a.
 //
 // A work unit is a 128-row query tile of one query head against the key tiles its
 // rows can see (global: all earlier keys; local: the last W keys; "Visual guide to
-// Gemma 4", section "Interleaving Layers"). Fully masked key tiles are never loaded;
-// only tiles that straddle the diagonal, the window edge or a sequence end are masked.
+// Gemma 4", section "Interleaving Layers"; bidirectional: every key of the sequence,
+// section "Vision encoder"). Fully masked key tiles are never loaded; only tiles that
+// straddle the diagonal, the window edge or a sequence end are masked.
 //
-// Roles (192 threads per CTA):
-//   warp 0     TMA producer: the Q tile once, then 16 KB stages of K and V through a
-//              ring (128-byte swizzle).
+// Roles (320 threads per CTA):
+//   warp 0     TMA producer: the Q tile once per unit, then stages of K and V (16 KB, or
+//              32 KB for the paired form at head dims >= 256) through a ring (128-byte
+//              swizzle).
 //   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score buffers
 //              (tcgen05.mma, both operands in shared memory), then O += P V with P read
 //              from TMEM and V from the ring.
-//   warps 2-5  softmax: one query row per thread; online softmax in fp32 with the
-//              running max only raised when it grows by more than 2^8, P written back to
-//              TMEM as bf16 over the scores, epilogue O / l.
+//   warps 2-9  softmax: two warps per TMEM lane quadrant, each taking one query row per
+//              lane and half of the score tile's columns; online softmax in fp32 with the
+//              running max only raised when it grows by more than 2^8 (the halves agree
+//              on the tile maximum through shared memory), P written back to TMEM as
+//              bf16 over the scores, epilogue O / l.
 // The MMA order is S(j), PV(j-1), S(j+1), PV(j), ... so the tensor core works on
 // S(j+1) while the softmax warps turn S(j) into P(j). The kernel is persistent: each
 // CTA (pair) stays resident and walks a list of work units, so barrier setup, TMEM
