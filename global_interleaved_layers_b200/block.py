@@ -1,7 +1,7 @@
 """Interleaved block runner: the attention calls of a block of layers as one CUDA graph.
 
 Gemma-4-style models interleave several sliding-window layers with one global layer
-("Visual guide to Gemma 4", section "Interleaved local and global attention": the 4:1
+("Visual guide to Gemma 4", section "Interleaving Layers": the 4:1
 and 5:1 patterns, the last layer of a block global). Each layer's prefill is two launches
 (rotated side copy, attention); a block of five layers is ten launches whose gaps the
 GPU otherwise spends idle between kernels. `InterleavedBlock` records the calls once and

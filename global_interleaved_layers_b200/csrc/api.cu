@@ -120,6 +120,52 @@ PrefillLayout prefill_layout(const gemma_attn_params* p, int64_t T) {
 }
 
 }  // namespace
+
+void set_launch_count(int n) { t_launches = n; }
+
+int decode_prepare(const gemma_attn_params* params, const void* q, const void* new_k, const void* new_v,
+                   const void* k_cache, const void* v_cache, int32_t cache_layout, int32_t cache_capacity,
+                   const int32_t* cache_seqlens, int32_t batch, int32_t n_q, int32_t max_cache_len,
+                   int32_t num_splits, DecodeArgs* a) {
+  int rc = check_params(params);
+  if (rc != GEMMA_ATTN_OK) return rc;
+  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
+  const bool global = params->kind == GEMMA_ATTN_GLOBAL;
+  if (!q || !new_k || !k_cache || !cache_seqlens) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (batch < 1 || n_q < 1 || num_splits < 1 || max_cache_len < 0) return GEMMA_ATTN_ERR_INVALID_ARG;
+  const bool keys_rotated = (cache_layout & GEMMA_ATTN_CACHE_KEYS_ROTATED) != 0;
+  if (keys_rotated && global) return GEMMA_ATTN_ERR_INVALID_ARG;  // the K=V tensor is also the values
+  cache_layout &= ~GEMMA_ATTN_CACHE_KEYS_ROTATED;
+  if (cache_layout != GEMMA_ATTN_CACHE_CONTIGUOUS && cache_layout != GEMMA_ATTN_CACHE_RING)
+    return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (cache_layout == GEMMA_ATTN_CACHE_RING && (global || cache_capacity != params->window))
+    return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (cache_layout == GEMMA_ATTN_CACHE_CONTIGUOUS && cache_capacity < max_cache_len)
+    return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (cache_capacity < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
+  const int group = params->num_q_heads / params->num_kv_heads;
+  if (group * n_q > decode_max_rows(params->head_dim)) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
+    return GEMMA_ATTN_ERR_MISALIGNED;
+  *a = DecodeArgs{};
+  a->q = static_cast<const uint16_t*>(q);
+  a->new_k = static_cast<const uint16_t*>(new_k);
+  a->new_v = static_cast<const uint16_t*>(new_v);
+  a->k_cache = static_cast<const uint16_t*>(k_cache);
+  a->v_cache = static_cast<const uint16_t*>(v_cache);
+  a->cache_seqlens = cache_seqlens;
+  a->batch = batch; a->n_q = n_q; a->num_q_heads = params->num_q_heads; a->num_kv_heads = params->num_kv_heads;
+  a->head_dim = params->head_dim; a->is_local = global ? 0 : 1; a->window = global ? 0 : params->window;
+  a->ring = cache_layout == GEMMA_ATTN_CACHE_RING; a->capacity = cache_capacity; a->num_splits = num_splits;
+  a->keys_rotated = keys_rotated ? 1 : 0;
+  a->r = rotated_pairs(params->rope_p, params->head_dim);
+  a->log2_base = log2((double)params->rope_base);
+  a->softmax_scale = params->softmax_scale;
+  if (!decode_supported(*a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
+  return GEMMA_ATTN_OK;
+}
+
 }  // namespace gattn
 
 using namespace gattn;
@@ -329,43 +375,12 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
                       const int32_t* cache_seqlens, int32_t batch, int32_t n_q, int32_t max_cache_len,
                       float* partial_o, float* partial_lse, int32_t num_splits, void* stream_) {
   t_launches = 0;
-  int rc = check_params(params);
-  if (rc != GEMMA_ATTN_OK) return rc;
-  if (params->kind == GEMMA_ATTN_BIDIR) return GEMMA_ATTN_ERR_UNSUPPORTED;  // prefill only
-  const bool global = params->kind == GEMMA_ATTN_GLOBAL;
-  if (!q || !new_k || !k_cache || !cache_seqlens || !partial_o || !partial_lse) return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (global != (new_v == nullptr) || global != (v_cache == nullptr)) return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (batch < 1 || n_q < 1 || num_splits < 1 || max_cache_len < 0) return GEMMA_ATTN_ERR_INVALID_ARG;
-  const bool keys_rotated = (cache_layout & GEMMA_ATTN_CACHE_KEYS_ROTATED) != 0;
-  if (keys_rotated && global) return GEMMA_ATTN_ERR_INVALID_ARG;  // the K=V tensor is also the values
-  cache_layout &= ~GEMMA_ATTN_CACHE_KEYS_ROTATED;
-  if (cache_layout != GEMMA_ATTN_CACHE_CONTIGUOUS && cache_layout != GEMMA_ATTN_CACHE_RING)
-    return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (cache_layout == GEMMA_ATTN_CACHE_RING && (global || cache_capacity != params->window))
-    return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (cache_layout == GEMMA_ATTN_CACHE_CONTIGUOUS && cache_capacity < max_cache_len)
-    return GEMMA_ATTN_ERR_INVALID_ARG;
-  if (cache_capacity < 1) return GEMMA_ATTN_ERR_INVALID_ARG;
-  const int group = params->num_q_heads / params->num_kv_heads;
-  if (group * n_q > decode_max_rows(params->head_dim)) return GEMMA_ATTN_ERR_UNSUPPORTED;
-  if (((uintptr_t)q | (uintptr_t)new_k | (uintptr_t)new_v | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u)
-    return GEMMA_ATTN_ERR_MISALIGNED;
+  if (!partial_o || !partial_lse) return GEMMA_ATTN_ERR_INVALID_ARG;
   DecodeArgs a{};  // out == nullptr: the kernel writes the split partials
-  a.q = static_cast<const uint16_t*>(q);
-  a.new_k = static_cast<const uint16_t*>(new_k);
-  a.new_v = static_cast<const uint16_t*>(new_v);
-  a.k_cache = static_cast<const uint16_t*>(k_cache);
-  a.v_cache = static_cast<const uint16_t*>(v_cache);
-  a.cache_seqlens = cache_seqlens;
+  const int rc = decode_prepare(params, q, new_k, new_v, k_cache, v_cache, cache_layout, cache_capacity,
+                                cache_seqlens, batch, n_q, max_cache_len, num_splits, &a);
+  if (rc != GEMMA_ATTN_OK) return rc;
   a.partial_o = partial_o; a.partial_lse = partial_lse;
-  a.batch = batch; a.n_q = n_q; a.num_q_heads = params->num_q_heads; a.num_kv_heads = params->num_kv_heads;
-  a.head_dim = params->head_dim; a.is_local = global ? 0 : 1; a.window = global ? 0 : params->window;
-  a.ring = cache_layout == GEMMA_ATTN_CACHE_RING; a.capacity = cache_capacity; a.num_splits = num_splits;
-  a.keys_rotated = keys_rotated ? 1 : 0;
-  a.r = rotated_pairs(params->rope_p, params->head_dim);
-  a.log2_base = log2((double)params->rope_base);
-  a.softmax_scale = params->softmax_scale;
-  if (!decode_supported(a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   if (launch_decode(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
   t_launches = 1;
   return GEMMA_ATTN_OK;

@@ -49,6 +49,9 @@ __global__ void cache_append_kernel(AppendArgs a) {
     if (lane == 0) atomicOr(&g_status, kStatusSeqlen);
     return;
   }
+  // A ring keeps the newest `capacity` positions: with more new tokens than slots, token
+  // i and token i + capacity map to the same slot, and only the later one is written.
+  if (a.ring && i < a.n_q - a.capacity) return;
   const int slot = a.ring ? pos % a.capacity : pos;
   const size_t src_row = (((size_t)b * a.n_q + i) * a.num_kv_heads + kvh) * a.head_dim;
   const size_t dst_row = (((size_t)b * a.num_kv_heads + kvh) * a.capacity + slot) * a.head_dim;

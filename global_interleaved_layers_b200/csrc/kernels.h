@@ -119,3 +119,18 @@ struct AppendArgs {
 cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream);
 
 }  // namespace gattn
+
+struct gemma_attn_params;
+
+namespace gattn {
+
+// Argument checks and DecodeArgs set-up shared by the decode entry points: fills every
+// field except the partial / final output pointers; returns a GEMMA_ATTN_* status.
+int decode_prepare(const gemma_attn_params* params, const void* q, const void* new_k, const void* new_v,
+                   const void* k_cache, const void* v_cache, int32_t cache_layout, int32_t cache_capacity,
+                   const int32_t* cache_seqlens, int32_t batch, int32_t n_q, int32_t max_cache_len,
+                   int32_t num_splits, DecodeArgs* a);
+// The count gemma_attn_last_launch_count reports for this host thread.
+void set_launch_count(int n);
+
+}  // namespace gattn

@@ -238,6 +238,9 @@ int gemma_attn_decode_noalloc(const gemma_attn_params* params, const void* q, co
  *   Order: call it after the decode / verify step that read these tokens from new_k /
  *   new_v. In a W-slot ring the new rows overwrite the slots of positions p - W, which
  *   that step's earlier queries still see (p - W > position - W for a query before p).
+ *   A ring holds the newest window positions: when n_q > cache_capacity, only the last
+ *   cache_capacity new tokens of a sequence are written (an earlier token's slot belongs
+ *   to a later one), so the result does not depend on the order the rows are written in.
  *   Errors: GEMMA_ATTN_ERR_INVALID_ARG / _MISALIGNED as gemma_attn_decode, before any
  *   launch. A contiguous-cache position p >= cache_capacity (or a negative length) writes
  *   nothing for that row and records GEMMA_ATTN_ERR_SEQLEN in the device status word,

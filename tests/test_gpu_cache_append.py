@@ -9,7 +9,8 @@ gemma_attn_cache_append writes the new tokens' rows into a decode cache. Checked
   - a full decode loop: decode token t (new rows beside the cache), append, decode token
     t + 1 from the extended cache -- each step equals the oracle over the whole history,
     including steps where the ring wraps;
-  - a contiguous cache without room records GEMMA_ATTN_ERR_SEQLEN and writes nothing.
+  - a contiguous cache without room records GEMMA_ATTN_ERR_SEQLEN and writes nothing;
+  - more new tokens than ring slots: the ring holds the newest window positions.
 """
 import numpy as np
 import pytest
@@ -162,3 +163,33 @@ def test_append_without_room_records_seqlen_and_writes_nothing():
     np.testing.assert_array_equal(got[0, :, 4], nk_h[0, 1])
     np.testing.assert_array_equal(got[1, :, 9], nk_h[1, 0])
     assert not got[1, :, :9].any() and not got[0, :, 5:].any()
+
+
+@pytest.mark.parametrize("rotated", [False, True])
+def test_ring_append_with_more_tokens_than_slots_keeps_the_newest(rotated):
+    """n_q > window: tokens i and i + W share a slot; the ring must end up holding the
+    newest W positions (what ring_from_history builds from the whole history)."""
+    layer = W.LayerSpec(W.LOCAL, 4, 2, 128, window=8, rope_p=1.0, rope_base=1e4)
+    B, Hkv, d, cap, n_q = 2, 2, 128, 8, 19
+    start = [5, 30]
+    k_hist = [W.normal_bf16(51 + b, 1, (start[b] + n_q, Hkv, d)) for b in range(B)]
+    v_hist = [W.normal_bf16(51 + b, 2, (start[b] + n_q, Hkv, d)) for b in range(B)]
+    k_src = [(_rotate_rows(k_hist[b], layer, range(start[b] + n_q)) if rotated else k_hist[b]) for b in range(B)]
+    kc0 = np.stack([ring_from_history(k_src[b][:start[b]], cap) for b in range(B)])
+    vc0 = np.stack([ring_from_history(v_hist[b][:start[b]], cap) for b in range(B)])
+    kc, vc = dev_bf16(kc0), dev_bf16(vc0)
+    nk = np.stack([k_hist[b][start[b]:] for b in range(B)])
+    nv = np.stack([v_hist[b][start[b]:] for b in range(B)])
+    lay = G.CACHE_RING | (G.CACHE_KEYS_ROTATED if rotated else 0)
+    G.gemma_attn_cache_append(_params(layer), dev_bf16(nk), dev_bf16(nv), kc, vc, lay, cap, dev_i32(start), B, n_q)
+    G.gemma_attn_check()
+    for b in range(B):
+        np.testing.assert_array_equal(host_bits(vc)[b], ring_from_history(v_hist[b], cap))
+        want_k = ring_from_history(k_src[b], cap)
+        got_k = host_bits(kc)[b]
+        if rotated:  # fp32 rotation against the oracle's fp64 one, then bf16: within one ulp
+            g = W.bf16_bits_to_f32(got_k).astype(np.float64)
+            w = W.bf16_bits_to_f32(want_k).astype(np.float64)
+            assert np.all(np.abs(g - w) <= np.maximum(np.abs(g), np.abs(w)) * 2.0 ** -7)
+        else:
+            np.testing.assert_array_equal(got_k, want_k)

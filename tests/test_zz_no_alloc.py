@@ -66,6 +66,7 @@ def test_noalloc_decode_matches_regular_path_twice(layer, cache_lens, n_q, ring,
         out = torch.empty((B, n_q, Hq, d), dtype=torch.float32, device="cuda")
         lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
         G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, splits, out, lse)
+        assert G.gemma_attn_last_launch_count() == 2  # the decode kernel, then the combine
         G.gemma_attn_check()
         assert_close(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), f"noalloc call {call}")
         np.testing.assert_allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), atol=1e-2, rtol=0)
@@ -114,6 +115,7 @@ def test_noalloc_single_split_writes_the_combined_result_directly(layer, cache_l
     out = torch.full((B, n_q, Hq, d), float("nan"), dtype=tdt, device="cuda")
     lse = torch.full((rows,), float("nan"), dtype=torch.float32, device="cuda")
     G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, 1, out, lse)
+    assert G.gemma_attn_last_launch_count() == 1  # the decode kernel alone
     out_nolse = torch.full_like(out, float("nan"))
     G.gemma_attn_decode_noalloc(p, q, nk, nv, kc, vc, layout, cap, lens, B, n_q, max_len, 1, out_nolse, None)
     G.gemma_attn_check()
