@@ -84,6 +84,33 @@ def test_31b_block_global_layer():
     _prefill_case(wl.layers[-1], wl.seq_lens, seed=200, rows=rows)
 
 
+def test_31b_block_global_layer_every_query_head():
+    """Sampled rows of all 32 query heads (every KV head's group), not only KV head 0's."""
+    layer = W.b31_block().layers[-1]
+    T = 32768
+    Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+    rows = np.array(sorted({0, 1, 127, 128, 4095, 16384, 32766, 32767} |
+                           set(int(x) for x in np.random.default_rng(2).integers(0, T, 4))), np.int32)
+    cu = np.array([0, T], np.int32)
+    pos = np.arange(T, dtype=np.int32)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(210)
+    q = torch.randn((T, Hq, d), generator=gen, device="cuda").to(torch.bfloat16)
+    k_host = W.normal_bf16(210, 1, (T, Hkv, d))
+    q_rows = W.normal_bf16(210, 0, (rows.shape[0], Hq, d))
+    ridx = torch.from_numpy(rows.astype(np.int64)).cuda()
+    q[ridx] = dev_bf16(q_rows)
+    out, _ = run_prefill(G, layer, q, dev_bf16(k_host), None, pos, cu, out_f32=True)
+    got = out[ridx].cpu().numpy()
+    del q, out
+    torch.cuda.empty_cache()
+    qo = np.zeros((T, Hq, d), np.uint16)  # only the sampled rows are read
+    qo[rows] = q_rows
+    ref, _ = oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                              qo, k_host, None, pos, cu, rows=rows)
+    assert_close(got, ref, "31B global layer, every query head")
+
+
 def test_31b_block_local_layer():
     wl = W.b31_block()
     _prefill_case(wl.layers[0], wl.seq_lens, seed=201)

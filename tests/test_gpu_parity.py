@@ -130,6 +130,35 @@ def test_prefill_shapes(layer, lens):
     _check_prefill(layer, lens, seed=3)
 
 
+# The single-CTA kernel at head dims >= 128: it runs when a query head has no partner that
+# shares its KV head (an odd GQA group: 1 or 3 query heads per KV head here), and for every
+# group when GEMMA_ATTN_NO_PAIR=1 is set (GQA mapping: "Visual guide to Gemma 4", section
+# "GQA").
+@pytest.mark.parametrize("layer,lens", [
+    (W.LayerSpec(W.LOCAL, 3, 3, 128, window=200, rope_p=1.0, rope_base=1e4), (300, 129)),
+    (W.LayerSpec(W.LOCAL, 3, 1, 256, window=300, rope_p=1.0, rope_base=1e4), (1, 400, 257)),
+    (W.LayerSpec(W.LOCAL, 2, 2, 512, window=150, rope_p=0.25, rope_base=1e4), (333,)),
+    (W.LayerSpec(W.GLOBAL, 1, 1, 128, rope_p=0.25, rope_base=1e6), (390, 7)),
+    (W.LayerSpec(W.GLOBAL, 3, 3, 256, rope_p=0.25, rope_base=1e4), (260, 1)),
+    (W.LayerSpec(W.GLOBAL, 3, 1, 512, rope_p=0.25, rope_base=1e6), (1, 200, 333)),
+])
+def test_prefill_single_cta_kernel_odd_group(layer, lens):
+    _check_prefill(layer, lens, seed=6)
+
+
+@pytest.mark.parametrize("layer,lens", [
+    (W.LayerSpec(W.LOCAL, 4, 2, 256, window=512, rope_p=1.0, rope_base=1e4), (1, 129, 300, 513)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 128, window=200, rope_p=1.0, rope_base=1e4), (450,)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6), (1, 200, 257)),
+    (W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.0, rope_base=1e6), (300,)),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 256, rope_p=0.25, rope_base=1e4), (390,)),
+])
+def test_prefill_even_group_on_the_single_cta_kernel(layer, lens, monkeypatch):
+    # the library reads the variable at every call
+    monkeypatch.setenv("GEMMA_ATTN_NO_PAIR", "1")
+    _check_prefill(layer, lens, seed=3)
+
+
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_prefill_output_only_16_byte_aligned(out_f32):
     # 32-byte output stores are used only where the output allows them; a 16-byte aligned
