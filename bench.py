@@ -1,13 +1,16 @@
 """Benchmark of the Gemma-4-style interleaved attention path on B200.
 
-A step is one pass of the hot path over the E2B-shaped prefill block: L = 8192 tokens,
-4 sliding-window layers (W = 512, 8/4 heads, d = 256) and 1 global layer (8/1 heads,
+A step is one pass of the hot path over the 31B-shaped prefill block: L = 32768 tokens,
+5 sliding-window layers (W = 1024, 32/16 heads, d = 256) and 1 global layer (32/4 heads,
 d = 512, K=V, p-RoPE p = 0.25). `value` is unmasked prefill TFLOP/s of that block, its
-ten launches (rotated side copy + attention per layer) replayed as one CUDA graph; the
-same calls launched one by one are reported as per_kind.e2b_block_eager.
+twelve launches (rotated side copy + attention per layer) replayed as one CUDA graph; the
+same calls launched one by one are reported as per_kind.b31_block_eager, and the
+E2B-shaped block (L = 8192, 4 local + 1 global) and the ragged 16-sequence 31B-shaped
+batch (both layer kinds) beside them.
 In the same run the decode path (split-KV + combine) is timed on the long-context
 decode shape (batch 8, 32/4 heads, global K=V cache of 131072 tokens at d = 512;
-local 1024-slot ring at d = 256, 32/16 heads) and reported in HBM GB/s.
+local 1024-slot ring at d = 256, 32/16 heads) and the 4-token verify of the ragged
+batch, reported in HBM GB/s.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Under torchrun each rank runs an independent replica (weak scaling); rank 0 prints
@@ -35,11 +38,11 @@ METRIC = "prefill TFLOP/s (unmasked FLOPs) and decode HBM GB/s per layer kind, %
 L2_FLUSH_BYTES = 256 << 20
 
 
-# DRAM bytes (read + write) per launch of prefill_kernel<512> on the E2B global layer, from the
-# ncu capture summarised in profiles/prefill_kernel_d512_e2b_global.md. Reported only while the
+# DRAM bytes (read + write) per launch of the global layer's attention kernel on the
+# headline block, from an ncu capture (see the profile summaries). Reported only while the
 # kernel's sources (their code: comments and blank lines do not count) still hash to the
 # captured state; any change makes it null until re-captured.
-NCU_TRAFFIC = {"bytes": 109307136, "sources_sha256_16": "169790a11edd9117",
+NCU_TRAFFIC = {"bytes": None, "sources_sha256_16": "",
                "sources": ["global_interleaved_layers_b200/csrc/prefill.cu",
                            "global_interleaved_layers_b200/csrc/common.cuh",
                            "global_interleaved_layers_b200/csrc/tile_plan.h",
@@ -195,14 +198,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
 
-def sample_rows(L: int, n_rand: int, seed: int = 1):
+def sample_rows(L: int, n_first: int, n_last: int, n_rand: int, seed: int = 1):
+    """First n_first, last n_last and n_rand rows from default_rng(seed), sorted, unique."""
     rng = np.random.default_rng(seed)
-    rows = set(range(min(128, L))) | set(range(max(0, L - 128), L))
+    rows = set(range(min(n_first, L))) | set(range(max(0, L - n_last), L))
     rows |= set(int(x) for x in rng.integers(0, L, size=n_rand))
     return np.array(sorted(rows), dtype=np.int32)
 
 
 def oracle_sample_flops(layer: W.LayerSpec, rows: np.ndarray) -> int:
+    """Unmasked FLOPs of the sampled query rows (one sequence, positions 0 .. L-1)."""
     pairs = 0
     for i in rows.tolist():
         vis = i + 1 if layer.kind == W.GLOBAL else min(i + 1, layer.window)
@@ -210,30 +215,66 @@ def oracle_sample_flops(layer: W.LayerSpec, rows: np.ndarray) -> int:
     return 4 * layer.head_dim * layer.num_q_heads * pairs
 
 
-def cpu_baseline(wl: W.PrefillWorkload, n_rand: int = 256):
-    """Time the fp64 oracle on a bounded row sample of every layer of the block."""
-    import oracle
-    oracle.build()
-    L = wl.total_tokens
-    rows = sample_rows(L, n_rand)
-    pos = wl.positions()
-    cu = wl.cu_seqlens()
-    flops = 0
-    elapsed = 0.0
-    done = set()
-    for li, layer in enumerate(wl.layers):
-        key = (layer.kind, layer.window, layer.head_dim, layer.num_q_heads, layer.num_kv_heads)
-        q, k, v = W.layer_inputs(layer, L, wl.seed, li)
-        t0 = time.perf_counter()
-        oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
-                         q, k, v, pos, cu, rows=rows)
-        elapsed += time.perf_counter() - t0
-        flops += oracle_sample_flops(layer, rows)
-        done.add(key)
-    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(rows)} query rows (first 128, last 128, {n_rand} from default_rng(1)) x all heads "
-                      f"of each of the {len(wl.layers)} layers, fp64 C oracle with OpenMP",
-            "seconds": elapsed}
+class OracleBlockSample:
+    """The fp64 oracle on a bounded row sample of each distinct layer shape of a block.
+
+    Inputs: every key/value row (the sampled rows see any of them) and only the sampled
+    query rows (the rest of q is never read: a zero array whose pages stay untouched)."""
+
+    def __init__(self, wl: W.PrefillWorkload, rows: np.ndarray):
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.wl = wl
+        self.rows = rows
+        L = wl.total_tokens
+        self.pos, self.cu = wl.positions(), wl.cu_seqlens()
+        self.kinds = []  # (layer, count in the block, q, k, v)
+        seen = {}
+        for li, layer in enumerate(wl.layers):
+            if layer in seen:
+                seen[layer][1] += 1
+                continue
+            base = wl.seed + 16 * li
+            q = np.zeros((L, layer.num_q_heads, layer.head_dim), np.uint16)
+            q[rows] = W.normal_bf16(base, 0, (rows.shape[0], layer.num_q_heads, layer.head_dim))
+            k = W.normal_bf16(base, 1, (L, layer.num_kv_heads, layer.head_dim))
+            v = None if layer.k_eq_v else W.normal_bf16(base, 2, (L, layer.num_kv_heads, layer.head_dim))
+            seen[layer] = [layer, 1, q, k, v]
+        self.kinds = list(seen.values())
+
+    def run(self):
+        """Time one pass over each distinct layer shape; returns (seconds for the block's
+        layers, each distinct shape's time counted once per layer of that shape, FLOPs of
+        that much work, query-row x head units)."""
+        sec = flops = units = 0
+        for layer, count, q, k, v in self.kinds:
+            t0 = time.perf_counter()
+            self.oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
+                                  q, k, v, self.pos, self.cu, rows=self.rows)
+            sec += count * (time.perf_counter() - t0)
+            flops += count * oracle_sample_flops(layer, self.rows)
+            units += count * self.rows.shape[0] * layer.num_q_heads
+        return sec, flops, units
+
+
+def cpu_baseline(wl: W.PrefillWorkload):
+    """The fp64 oracle on a bounded row sample of the headline block (about 10 s on 16
+    host cores): its FLOP rate, query rows per second, and the full block's time
+    extrapolated from that rate."""
+    rows = sample_rows(wl.total_tokens, 32, 32, 64)
+    smp = OracleBlockSample(wl, rows)
+    sec, flops, units = smp.run()
+    rate = flops / sec
+    block_flops = sum(W.prefill_flops(wl.seq_lens, layer) for layer in wl.layers)
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": smp.oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} query rows (first 32, last 32, 64 from default_rng(1)) x all heads of "
+                      f"each distinct layer shape of {wl.name}; the local shape's time counted once per local "
+                      f"layer ({sum(1 for ly in wl.layers if ly.kind == W.LOCAL)} of them); fp64 C oracle with "
+                      "OpenMP",
+            "seconds": sec, "query_rows_per_s": units / sec, "query_rows_unit": "query row x head",
+            "extrapolated_full_block_s": block_flops / rate,
+            "extrapolated_note": "extrapolated: the full block's unmasked FLOPs / the sample's FLOP rate"}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -246,43 +287,32 @@ def dist_setup(n_gpus: int):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, each step a bounded sample of
+    the headline block (its first 16 and last 16 query rows of every layer shape)."""
     world, rank, local = dist_setup(args.gpus)
     if rank != 0:
         return
-    import oracle
-    oracle.build()
-    wl = W.e2b_block()
+    wl = W.b31_block()
     L = wl.total_tokens
-    pos, cu = wl.positions(), wl.cu_seqlens()
-    inputs = [W.layer_inputs(layer, L, wl.seed, li) for li, layer in enumerate(wl.layers)]
-    rows = sample_rows(L, 0)[:64]  # a bounded sample per step (first 64 rows) keeps each step to seconds
-    rows = np.concatenate([rows, np.arange(L - 64, L, dtype=np.int32)])
-
-    def step():
-        f = 0
-        for li, layer in enumerate(wl.layers):
-            q, k, v = inputs[li]
-            oracle.attention(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
-                             q, k, v, pos, cu, rows=rows)
-            f += oracle_sample_flops(layer, rows)
-        return f
-
+    rows = sample_rows(L, 16, 16, 0)
+    smp = OracleBlockSample(wl, rows)
     for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    flops = 0
+        smp.run()
+    sec = flops = 0
     for _ in range(args.steps):
-        flops += step()
-    el = time.perf_counter() - t0
-    value = flops / el / 1e12
-    sample = (f"{len(rows)} query rows (first 64, last 64) x all heads of each layer of the E2B block per step, "
-              "fp64 C oracle with OpenMP")
+        s_, f_, _ = smp.run()
+        sec += s_
+        flops += f_
+    value = flops / sec / 1e12
+    sample = (f"{len(rows)} query rows (first 16, last 16) x all heads of each distinct layer shape of {wl.name} "
+              "per step, the local shape's time counted once per local layer; fp64 C oracle with OpenMP")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L, "layers": "4 local (W=512) + 1 global"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L,
+                   "layers": "5 local (W=1024, 32/16 heads, d=256) + 1 global (32/4 heads, d=512, K=V, p=0.25)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": smp.oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -290,16 +320,133 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+class BlockBench:
+    """One prefill block's device buffers and its timings (graph replay and call by call)."""
+
+    def __init__(self, G, torch, dev, wl: W.PrefillWorkload, seed: int):
+        self.G, self.torch, self.wl = G, torch, wl
+        L = wl.total_tokens
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        self.layers = []
+        max_ws = 0
+        for li, layer in enumerate(wl.layers):
+            q = torch.randn((L, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+            k = torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+            v = None if layer.k_eq_v else torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen,
+                                                     device=dev).to(torch.bfloat16)
+            out = torch.empty_like(q)
+            p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
+                         rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
+            max_ws = max(max_ws, G.gemma_attn_prefill_workspace_size(p, L))
+            self.layers.append(dict(spec=layer, q=q, k=k, v=v, out=out, p=p,
+                                    flops=W.prefill_flops(wl.seq_lens, layer)))
+        self.ws = torch.empty(max(max_ws, 256), dtype=torch.uint8, device=dev)
+        self.pos = torch.from_numpy(wl.positions()).to(dev)
+        self.cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
+        self.total_flops = sum(ly["flops"] for ly in self.layers)
+        self.glob = [li for li, ly in enumerate(self.layers) if ly["spec"].kind == W.GLOBAL]
+        self.loc = [li for li, ly in enumerate(self.layers) if ly["spec"].kind == W.LOCAL]
+        self.blk = None
+
+    def call_args(self, li, stream):
+        ly = self.layers[li]
+        S = len(self.wl.seq_lens)
+        L = self.wl.total_tokens
+        return (ly["p"], ly["q"], ly["k"], ly["v"], ly["out"], None, self.pos, self.cu, S, L,
+                max(self.wl.seq_lens), self.ws, self.ws.numel(), stream)
+
+    def run_layer(self, li, stream):
+        # one layer = the prefill's two phases back to back (exactly what gemma_attn_prefill runs)
+        G = self.G
+        call = self.call_args(li, stream)
+        G.gemma_attn_prefill_rotate(*call)
+        n = G.gemma_attn_last_launch_count()
+        G.gemma_attn_prefill_attend(*call)
+        return n + G.gemma_attn_last_launch_count()
+
+    def capture(self, stream, warmup):
+        """The block's launches recorded once as a CUDA graph, with two events around the
+        global layer's attention kernel (each recorded event costs the stream microseconds,
+        so there are no others)."""
+        torch, G = self.torch, self.G
+        from global_interleaved_layers_b200.block import BlockLayer, InterleavedBlock
+        S, L = len(self.wl.seq_lens), self.wl.total_tokens
+        self.blk = InterleavedBlock([BlockLayer(ly["p"], ly["q"], ly["k"], ly["v"], ly["out"], None, self.pos,
+                                                self.cu, S, L, max(self.wl.seq_lens), self.ws)
+                                     for ly in self.layers])
+        self.att0 = torch.cuda.Event(enable_timing=True, external=True)
+        self.att1 = torch.cuda.Event(enable_timing=True, external=True)
+        g0 = self.glob[0]
+        evs = [((None, self.att0, self.att1) if li == g0 else None) for li in range(len(self.layers))]
+        self.launches_per_step = self.blk.capture(events=evs)
+        for _ in range(warmup):
+            self.blk.replay()
+        torch.cuda.synchronize()
+        G.gemma_attn_check()
+
+    def time_graph(self, stream, steps, flush_l2):
+        """Per-step ms of graph replays (L2 flushed before each) and the global attention
+        kernel's ms inside each."""
+        torch = self.torch
+        step_ms, att_ms = [], []
+        for _ in range(steps):
+            flush_l2()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            self.blk.replay()
+            s1.record(stream)
+            # the graph's events are re-recorded by every replay: read them now
+            s1.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+            att_ms.append(self.att0.elapsed_time(self.att1))
+        self.G.gemma_attn_check()
+        return step_ms, att_ms
+
+    def release_graph(self):
+        if self.blk is not None:
+            self.blk.graph = None
+
+    def time_eager(self, stream, steps, flush_l2):
+        """The same step launched call by call (no graph), with events around every layer.
+        Returns (mean step ms, {layer index: mean ms})."""
+        torch = self.torch
+        step, per = [], {}
+        for _ in range(steps):
+            flush_l2()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            evs = []
+            for li in range(len(self.layers)):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                self.run_layer(li, stream)
+                e1.record(stream)
+                evs.append((e0, e1))
+            s1.record(stream)
+            torch.cuda.synchronize()
+            step.append(s0.elapsed_time(s1))
+            for li, (e0, e1) in enumerate(evs):
+                per.setdefault(li, []).append(e0.elapsed_time(e1))
+        self.G.gemma_attn_check()
+        return float(np.mean(step)), {li: float(np.mean(v)) for li, v in per.items()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="only the headline block (no per_kind extras)")
     ap.add_argument("--case", default="block",
-                    choices=["block", "global_prefill", "local_prefill", "global_decode", "local_decode"],
+                    choices=["block", "global_prefill", "local_prefill", "global_prefill_31b_h8",
+                             "global_decode", "local_decode", "global_verify"],
                     help="block: the benchmark (one JSON line). Any other value runs only that operation "
                          "(warmup + steps launches, no timing contract) for profiler captures.")
     ap.add_argument("--ctx", type=int, default=0, help="decode cases: cached tokens per sequence (0: 131072)")
@@ -323,6 +470,7 @@ def main():
     reps = Replicas(backend="nccl", timeout_s=120)  # process group only when WORLD_SIZE > 1
     dev = torch.device("cuda", local)
     peaks = measured_peaks()
+    peak_t = peaks["bf16_tflops"]  # burst: the kernels are timed in steps of tens of ms at full clock
 
     def barrier():
         reps.barrier()
@@ -341,156 +489,119 @@ def main():
         flush_buf.fill_(1.0)
         torch.sum(flush_read, dim=0, out=flush_sink)
 
-    # ------------------------------------------------------------------ prefill block inputs
-    wl = W.e2b_block()
-    L = wl.total_tokens
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1234 + rank)
-    layers = []
-    max_ws = 0
-    for li, layer in enumerate(wl.layers):
-        q = torch.randn((L, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
-        k = torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
-        v = None if layer.k_eq_v else torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen,
-                                                 device=dev).to(torch.bfloat16)
-        out = torch.empty_like(q)
-        p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, window=layer.window,
-                     rope_p=layer.rope_p, rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
-        ws_bytes = G.gemma_attn_prefill_workspace_size(p, L)
-        max_ws = max(max_ws, ws_bytes)
-        layers.append(dict(spec=layer, q=q, k=k, v=v, out=out, p=p, flops=W.prefill_flops(wl.seq_lens, layer)))
-    ws = torch.empty(max(max_ws, 256), dtype=torch.uint8, device=dev)
-    pos = torch.from_numpy(wl.positions()).to(dev)
-    cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
-    total_flops = sum(l["flops"] for l in layers)
-
     stream = torch.cuda.current_stream()
-    kind_ev = {}  # per layer index: the layer's time (ms) in each timed step
-    attend_ev = {}  # the same for its attention kernel alone
 
-    def run_layer(li):
-        # one layer = the prefill's two phases back to back (exactly what gemma_attn_prefill runs)
-        l = layers[li]
-        call = (l["p"], l["q"], l["k"], l["v"], l["out"], None, pos, cu, 1, L, L, ws, ws.numel(), stream)
-        G.gemma_attn_prefill_rotate(*call)
-        n = G.gemma_attn_last_launch_count()
-        G.gemma_attn_prefill_attend(*call)
-        return n + G.gemma_attn_last_launch_count()
-
-    def step():
-        n = 0
-        for li in range(len(layers)):
-            n += run_layer(li)
-        return n
-
-    log("prefill warmup")
+    # ------------------------------------------------------------------ headline: the 31B-shaped block
+    wl = W.b31_block()
+    L = wl.total_tokens
+    bb = BlockBench(G, torch, dev, wl, seed=1234 + rank)
+    log("31B block warmup")
     for _ in range(args.warmup):
-        step()
-    G.gemma_attn_check()
-    torch.cuda.synchronize()
-
-    # The timed step is the block's ten launches (rotate + attend per layer) recorded once
-    # as a CUDA graph and replayed (global_interleaved_layers_b200.block), as a serving
-    # loop runs a fixed-shape step. Two events inside the graph time the global layer's
-    # attention kernel (each recorded event costs the stream a few microseconds, so there
-    # are no others). The same calls launched one by one, with events around every layer,
-    # are timed after it (per_kind.e2b_block_eager and the per-layer figures).
-    from global_interleaved_layers_b200.block import BlockLayer, InterleavedBlock
-    blk = InterleavedBlock([BlockLayer(l["p"], l["q"], l["k"], l["v"], l["out"], None, pos, cu, 1, L, L, ws)
-                            for l in layers])
-    glob = [li for li, l in enumerate(layers) if l["spec"].kind == W.GLOBAL]
-    loc = [li for li, l in enumerate(layers) if l["spec"].kind == W.LOCAL]
-    att0 = torch.cuda.Event(enable_timing=True, external=True)
-    att1 = torch.cuda.Event(enable_timing=True, external=True)
-    gev = [((None, att0, att1) if li == glob[0] else None) for li in range(len(layers))]
-    launches_per_step = blk.capture(events=gev)
-    for _ in range(args.warmup):
-        blk.replay()
+        for li in range(len(bb.layers)):
+            bb.run_layer(li, stream)
     torch.cuda.synchronize()
     G.gemma_attn_check()
-    log("prefill timed")
-
-    step_events = []
-    launches = 0
+    bb.capture(stream, args.warmup)
+    log("31B block timed")
     with ClockSampler(local) as clocks:
         barrier()
         torch.cuda.synchronize()
-        for _ in range(args.steps):
-            flush_l2()
-            s0 = torch.cuda.Event(enable_timing=True)
-            s1 = torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            blk.replay()
-            s1.record(stream)
-            launches += launches_per_step
-            step_events.append((s0, s1))
-            # the graph's events are re-recorded by every replay: read them now
-            s1.synchronize()
-            attend_ev.setdefault(glob[0], []).append(att0.elapsed_time(att1))
+        step_ms, att_ms = bb.time_graph(stream, args.steps, flush_l2)
         torch.cuda.synchronize()
         barrier()
     clk = clocks.summary()
-    G.gemma_attn_check()
-    step_ms = [a.elapsed_time(b) for a, b in step_events]
+    launches = bb.launches_per_step * args.steps
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / args.steps
-    value = world * total_flops * args.steps / (total_ms * 1e-3) / 1e12
-    blk.graph = None  # release the graph before its buffers are reused below
+    value = world * bb.total_flops * args.steps / (total_ms * 1e-3) / 1e12
+    bb.release_graph()
 
-    # the same step launched call by call (no graph), with events around every layer
-    eager_events = []
-    layer_events = []
     barrier()
-    for _ in range(args.steps):
-        flush_l2()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        evs = []
-        for li in range(len(layers)):
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            run_layer(li)
-            e1.record(stream)
-            evs.append((e0, e1))
-        s1.record(stream)
-        eager_events.append((s0, s1))
-        layer_events.append(evs)
-    torch.cuda.synchronize()
-    G.gemma_attn_check()
+    eager_ms, per_layer_ms = bb.time_eager(stream, max(3, args.steps // 2), flush_l2)
+    eager_ms = max_over_ranks(eager_ms)
     barrier()
-    eager_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in eager_events])))
-    for evs in layer_events:
-        for li, (e0, e1) in enumerate(evs):
-            kind_ev.setdefault(li, []).append(e0.elapsed_time(e1))
-    block_eager = {"ms": eager_ms, "tflops": world * total_flops / (eager_ms * 1e-3) / 1e12,
-                   "launches": launches_per_step,
-                   "note": "the timed step's calls launched one by one from Python (no CUDA graph), "
-                           "with events around every layer (per_kind.local_prefill / global_prefill)"}
-
-    per_layer_ms = {li: float(np.mean(v)) for li, v in kind_ev.items()}
-    g_ms = float(np.mean([per_layer_ms[i] for i in glob]))
-    l_ms = float(np.mean([per_layer_ms[i] for i in loc]))
-    g_flops = layers[glob[0]]["flops"]
-    l_flops = layers[loc[0]]["flops"]
+    g_ms = float(np.mean([per_layer_ms[i] for i in bb.glob]))
+    l_ms = float(np.mean([per_layer_ms[i] for i in bb.loc]))
+    g_flops = bb.layers[bb.glob[0]]["flops"]
+    l_flops = bb.layers[bb.loc[0]]["flops"]
     g_tflops = g_flops / (g_ms * 1e-3) / 1e12
-    # the dominant kernel (the global layer's attention) per launch, timed inside the step
-    attend_ms = max_over_ranks(float(np.mean(attend_ev[glob[0]])))
-    attend_tflops = g_flops / (attend_ms * 1e-3) / 1e12
     l_tflops = l_flops / (l_ms * 1e-3) / 1e12
-    peak_t = peaks["bf16_tflops_sustained"]
-    loc_spec = layers[loc[0]]["spec"]
+    # the dominant kernel (the global layer's attention) per launch, timed inside the step
+    attend_ms = max_over_ranks(float(np.mean(att_ms)))
+    attend_tflops = g_flops / (attend_ms * 1e-3) / 1e12
+    loc_spec = bb.layers[bb.loc[0]]["spec"]
     local_ceiling = loc_spec.window / (loc_spec.window + 128 - 1)
+    per_kind = {
+        "local_prefill": {"tflops": l_tflops, "ms": l_ms, "frac_of_peak": l_tflops / peak_t,
+                          "tile_geometry_ceiling": local_ceiling,
+                          "shape": "31B local layer: L=32768, W=1024, 32/16 heads, d=256 (rotated copy + attention)"},
+        "global_prefill": {"tflops": g_tflops, "ms": g_ms, "frac_of_peak": g_tflops / peak_t,
+                           "shape": "31B global layer: L=32768, 32/4 heads, d=512, K=V, p=0.25 "
+                                    "(rotated copy + attention)"},
+        "b31_block_eager": {"ms": eager_ms, "tflops": world * bb.total_flops / (eager_ms * 1e-3) / 1e12,
+                            "launches": bb.launches_per_step,
+                            "note": "the timed step's calls launched one by one from Python (no CUDA graph), "
+                                    "with events around every layer (per_kind.local_prefill / global_prefill)"},
+    }
 
     # ------------------------------------------------------------------ e2e through host buffers
+    e2e = bench_e2e(G, torch, dev, stream, bb, args, world, max_over_ranks, barrier)
+    del bb
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------------ the other workloads
+    if not args.no_extra:
+        per_kind["e2b_block"] = bench_block_graph(G, torch, dev, stream, W.e2b_block(), args, world,
+                                                  max_over_ranks, barrier, flush_l2, peak_t)
+        per_kind.update(bench_ragged_prefill(G, torch, dev, stream, args, max_over_ranks, barrier, flush_l2, peak_t))
+        if not args.no_decode:
+            per_kind.update(bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks,
+                                         barrier))
+        per_kind["vision_bidir_prefill"] = bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world,
+                                                        max_over_ranks, barrier)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L,
+                   "layers": "5 local (W=1024, 32/16 heads, d=256) + 1 global (32/4 heads, d=512, K=V, p=0.25)",
+                   "l2": "inputs larger than L2, and L2 flushed before every timed step (256 MiB write, then a "
+                         "256 MiB read of another buffer, so no dirty lines are left for the step to write back); "
+                         "per-step CUDA events",
+                   "parallelism": f"replicas x{world}"},
+        "per_kind": per_kind,
+        "roofline": {"bound": "tensor", "achieved": attend_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": attend_tflops / peak_t, "kernel_ms": attend_ms, "traffic": ncu_traffic(),
+                     "traffic_unit": "bytes per launch",
+                     "frac_of_sustained_peak": attend_tflops / peaks["bf16_tflops_sustained"],
+                     "kernel": "prefill_kernel<512>: the 31B global layer's attention phase (35.19 TFLOP of "
+                               "unmasked work per launch), timed with CUDA events recorded inside the timed "
+                               "step's graph (per_kind.global_prefill, from the call-by-call run, also counts "
+                               "the rotated side copy)",
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)"},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        log("cpu baseline")
+        result["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    reps.close()
+
+
+def bench_e2e(G, torch, dev, stream, bb, args, world, max_over_ranks, barrier):
+    """The block through the public API with host buffers: every step copies each layer's
+    q/k/v from pinned host memory and its output back, inside the timed region."""
     host = []
     h2d = d2h = 0
-    for l in layers:
-        hq = l["q"].cpu().pin_memory()
-        hk = l["k"].cpu().pin_memory()
-        hv = None if l["v"] is None else l["v"].cpu().pin_memory()
-        ho = torch.empty(l["out"].shape, dtype=torch.bfloat16).pin_memory()
+    for ly in bb.layers:
+        hq = ly["q"].cpu().pin_memory()
+        hk = ly["k"].cpu().pin_memory()
+        hv = None if ly["v"] is None else ly["v"].cpu().pin_memory()
+        ho = torch.empty(ly["out"].shape, dtype=torch.bfloat16).pin_memory()
         host.append((hq, hk, hv, ho))
         h2d += hq.numel() * 2 + hk.numel() * 2 + (0 if hv is None else hv.numel() * 2)
         d2h += ho.numel() * 2
@@ -501,94 +612,117 @@ def main():
     # attention of another. Every step still moves all of its inputs and outputs.
     h2d_stream = torch.cuda.Stream(device=dev)
     d2h_stream = torch.cuda.Stream(device=dev)
-    nl = len(layers)
+    nl = len(bb.layers)
     ev_in = [torch.cuda.Event() for _ in range(nl)]
     ev_done = [torch.cuda.Event() for _ in range(nl)]
     ev_out = [torch.cuda.Event() for _ in range(nl)]
     first_step = [True]
 
     def e2e_step():
-        for li, l in enumerate(layers):
+        for li, ly in enumerate(bb.layers):
             hq, hk, hv, ho = host[li]
             with torch.cuda.stream(h2d_stream):
                 if not first_step[0]:
                     h2d_stream.wait_event(ev_done[li])  # the previous step's call has read the inputs
-                l["q"].copy_(hq, non_blocking=True)
-                l["k"].copy_(hk, non_blocking=True)
+                ly["q"].copy_(hq, non_blocking=True)
+                ly["k"].copy_(hk, non_blocking=True)
                 if hv is not None:
-                    l["v"].copy_(hv, non_blocking=True)
+                    ly["v"].copy_(hv, non_blocking=True)
                 ev_in[li].record(h2d_stream)
             stream.wait_event(ev_in[li])
             if not first_step[0]:
                 stream.wait_event(ev_out[li])  # the previous step's output has been read back
-            run_layer(li)
+            bb.run_layer(li, stream)
             ev_done[li].record(stream)
             with torch.cuda.stream(d2h_stream):
                 d2h_stream.wait_event(ev_done[li])
-                ho.copy_(l["out"], non_blocking=True)
+                ho.copy_(ly["out"], non_blocking=True)
                 ev_out[li].record(d2h_stream)
         first_step[0] = False
 
     log("e2e")
-    for _ in range(3):
+    for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e_steps = max(3, args.steps // 2)
+    e_steps = max(3, args.steps // 4)
     e0.record(h2d_stream)
     for _ in range(e_steps):
         e2e_step()
     e1.record(d2h_stream)  # after the last read-back, which follows every earlier operation
     torch.cuda.synchronize()
+    G.gemma_attn_check()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
-    e2e_value = world * total_flops / (e2e_ms * 1e-3) / 1e12
+    value = world * bb.total_flops / (e2e_ms * 1e-3) / 1e12
+    del host
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_ms, "steps": e_steps}
 
-    # ------------------------------------------------------------------ decode (long context)
-    decode = None
-    if not args.no_decode:
-        decode = bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier)
-    vision = bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier)
 
-    result = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": 1, "seq_len": L,
-                   "layers": "4 local (W=512, 8/4 heads, d=256) + 1 global (8/1 heads, d=512, K=V, p=0.25)",
-                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another "
-                          "buffer, so no dirty lines are left for the step to write back); per-step CUDA events",
-                   "parallelism": f"replicas x{world}"},
-        "per_kind": {
-            "local_prefill": {"tflops": l_tflops, "ms": l_ms, "frac_of_peak": l_tflops / peak_t,
-                              "tile_geometry_ceiling": local_ceiling},
-            "global_prefill": {"tflops": g_tflops, "ms": g_ms, "frac_of_peak": g_tflops / peak_t},
-            "e2b_block_eager": block_eager,
-        },
-        "roofline": {"bound": "tensor", "achieved": attend_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": attend_tflops / peak_t, "kernel_ms": attend_ms, "traffic": ncu_traffic(),
-                     "traffic_unit": "bytes per launch",
-                     "kernel": "prefill_kernel<512, 1>: the global layer's attention phase, timed with "
-                               "CUDA events recorded inside the timed step's graph (per_kind.global_prefill, from "
-                               "the call-by-call run, also counts the "
-                               "rotated side copy)",
-                     "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": launches,
-        "clocks": clk,
-    }
-    if decode is not None:
-        result["per_kind"].update(decode)
-    result["per_kind"]["vision_bidir_prefill"] = vision
-    if rank == 0 and not args.no_cpu_baseline:
-        log("cpu baseline")
-        result["cpu_baseline"] = cpu_baseline(wl)
-    if rank == 0:
-        print(json.dumps(result), flush=True)
-    reps.close()
+def bench_block_graph(G, torch, dev, stream, wl, args, world, max_over_ranks, barrier, flush_l2, peak_t):
+    """A block's step replayed as a CUDA graph (per_kind entry for a second block shape)."""
+    bb = BlockBench(G, torch, dev, wl, seed=77)
+    for li in range(len(bb.layers)):
+        bb.run_layer(li, stream)
+    torch.cuda.synchronize()
+    bb.capture(stream, args.warmup)
+    log(f"{wl.name} timed")
+    barrier()
+    step_ms, att_ms = bb.time_graph(stream, args.steps, flush_l2)
+    barrier()
+    ms = max_over_ranks(float(np.mean(step_ms)))
+    att = max_over_ranks(float(np.mean(att_ms)))
+    g_flops = bb.layers[bb.glob[0]]["flops"]
+    bb.release_graph()
+    res = {"ms": ms, "tflops": world * bb.total_flops / (ms * 1e-3) / 1e12, "launches": bb.launches_per_step,
+           "global_attention_ms": att, "global_attention_tflops": g_flops / (att * 1e-3) / 1e12,
+           "global_attention_frac_of_peak": g_flops / (att * 1e-3) / 1e12 / peak_t,
+           "shape": f"{wl.name}: " + ", ".join(sorted({str(ly['spec']) for ly in bb.layers}))}
+    del bb
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_ragged_prefill(G, torch, dev, stream, args, max_over_ranks, barrier, flush_l2, peak_t):
+    """The ragged 16-sequence 31B-shaped batch (229,704 tokens): one local and one global
+    layer's prefill, each call timed alone."""
+    pre, _ = W.ragged_31b()
+    bb = BlockBench(G, torch, dev, pre, seed=91)
+    res = {}
+    steps = max(3, args.steps // 4)
+    for li in range(len(bb.layers)):
+        spec = bb.layers[li]["spec"]
+        tag = "ragged_global_prefill" if spec.kind == W.GLOBAL else "ragged_local_prefill"
+        for _ in range(2):
+            bb.run_layer(li, stream)
+        torch.cuda.synchronize()
+        G.gemma_attn_check()
+        log(tag)
+        barrier()
+        evs = []
+        for _ in range(steps):
+            flush_l2()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            bb.run_layer(li, stream)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        G.gemma_attn_check()
+        barrier()
+        ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+        tf = bb.layers[li]["flops"] / (ms * 1e-3) / 1e12
+        res[tag] = {"tflops": tf, "ms": ms, "frac_of_peak": tf / peak_t, "steps": steps,
+                    "tflop_per_call": bb.layers[li]["flops"] / 1e12,
+                    "shape": f"16 sequences, {pre.total_tokens} tokens (lengths from default_rng(7)), {spec} "
+                             "(rotated copy + attention)"}
+    del bb
+    torch.cuda.empty_cache()
+    return res
 
 
 def bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
@@ -773,7 +907,7 @@ def bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_r
     ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
     flops = W.prefill_flops(wl.seq_lens, layer)
     tflops = flops / (ms * 1e-3) / 1e12
-    return {"tflops": tflops, "ms": ms, "frac_of_peak": tflops / peaks["bf16_tflops_sustained"],
+    return {"tflops": tflops, "ms": ms, "frac_of_peak": tflops / peaks["bf16_tflops"],
             "launches": 2, "shape": f"{len(wl.seq_lens)} images x {maxlen} patches, {layer.num_q_heads} heads, "
                                     f"d={layer.head_dim}, bidirectional, 2D RoPE (rotated copy + attention)"}
 
@@ -787,9 +921,16 @@ def run_case(args):
     stream = torch.cuda.current_stream()
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
-    if args.case.endswith("prefill"):
+    if "prefill" in args.case:
         wl = W.e2b_block()
         layer = wl.layers[-1] if args.case == "global_prefill" else wl.layers[0]
+        if args.case == "global_prefill_31b_h8":
+            # the 31B global layer's sequence length with a quarter of its heads (8 query heads,
+            # one KV head): DRAM traffic per launch scales with the heads, for a capture that
+            # stays small
+            wl = W.PrefillWorkload(name="31b_global_h8", seq_lens=(32768,), seed=0,
+                                   layers=(W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6),))
+            layer = wl.layers[0]
         L = wl.total_tokens
         q = torch.randn((L, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
         k = torch.randn((L, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
@@ -804,6 +945,28 @@ def run_case(args):
 
         def op():
             G.gemma_attn_prefill(p, q, k, v, out, None, pos, cu, 1, L, L, ws, ws_bytes, stream)
+    elif args.case == "global_verify":
+        _, ver = W.ragged_31b()
+        layer = ver.layers[0]
+        B, n_q = ver.batch, ver.n_q
+        Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+        cap = max(ver.cache_lens)
+        kc = torch.empty((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev).normal_(generator=gen)
+        q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+        nk = torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+        lens = torch.tensor(list(ver.cache_lens), dtype=torch.int32, device=dev)
+        p = G.params(layer.kind, Hq, Hkv, d, rope_p=layer.rope_p, rope_base=layer.rope_base,
+                     softmax_scale=layer.softmax_scale)
+        splits = G.gemma_attn_decode_num_splits(p, B, n_q, cap)
+        rows = B * n_q * Hq
+        po = torch.empty((splits, rows, d), dtype=torch.float32, device=dev)
+        pl = torch.empty((splits, rows), dtype=torch.float32, device=dev)
+        out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
+
+        def op():
+            G.gemma_attn_decode(p, q, nk, None, kc, None, G.CACHE_CONTIGUOUS, cap, lens, B, n_q, cap, po, pl, splits,
+                                stream)
+            G.gemma_attn_combine(po, pl, splits, rows, d, G.OUT_BF16, out, None, stream)
     else:
         wl = W.long_decode()
         layer = wl.layers[0] if args.case == "global_decode" else wl.layers[1]

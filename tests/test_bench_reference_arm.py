@@ -19,7 +19,7 @@ def test_reference_arm_prints_one_contract_line():
                 "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in r, key
     assert r["impl"] == "reference" and r["value"] > 0 and r["warmup"] >= 3
-    assert r["config"]["workload"] == "e2b_block_L8192"
+    assert r["config"]["workload"] == "31b_block_L32768"
     assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
     assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
     assert r["e2e"]["value"] == r["value"]
