@@ -123,6 +123,19 @@ PrefillLayout prefill_layout(const gemma_attn_params* p, int64_t T) {
 
 void set_launch_count(int n) { t_launches = n; }
 
+bool encode_cache_map(CUtensorMap* m, const void* base, int d, int capacity, int planes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)capacity, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * capacity * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int decode_prepare(const gemma_attn_params* params, const void* q, const void* new_k, const void* new_v,
                    const void* k_cache, const void* v_cache, int32_t cache_layout, int32_t cache_capacity,
                    const int32_t* cache_seqlens, int32_t batch, int32_t n_q, int32_t max_cache_len,
@@ -162,6 +175,8 @@ int decode_prepare(const gemma_attn_params* params, const void* q, const void* n
   a->r = rotated_pairs(params->rope_p, params->head_dim);
   a->log2_base = log2((double)params->rope_base);
   a->softmax_scale = params->softmax_scale;
+  a->q_pos_offset = nullptr;
+  a->new_keys = 1;
   if (!decode_supported(*a)) return GEMMA_ATTN_ERR_UNSUPPORTED;
   return GEMMA_ATTN_OK;
 }
@@ -380,6 +395,31 @@ int gemma_attn_decode(const gemma_attn_params* params, const void* q, const void
   const int rc = decode_prepare(params, q, new_k, new_v, k_cache, v_cache, cache_layout, cache_capacity,
                                 cache_seqlens, batch, n_q, max_cache_len, num_splits, &a);
   if (rc != GEMMA_ATTN_OK) return rc;
+  a.partial_o = partial_o; a.partial_lse = partial_lse;
+  if (launch_decode(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
+  t_launches = 1;
+  return GEMMA_ATTN_OK;
+}
+
+int gemma_attn_decode_shard(const gemma_attn_params* params, const void* q, const void* new_k, const void* k_cache,
+                            int32_t cache_capacity, const int32_t* shard_seqlens, const int32_t* q_pos_offset,
+                            int32_t include_new, int32_t batch, int32_t n_q, int32_t max_shard_len,
+                            float* partial_o, float* partial_lse, int32_t num_splits, void* stream_) {
+  t_launches = 0;
+  if (!params || params->kind != GEMMA_ATTN_GLOBAL) return GEMMA_ATTN_ERR_INVALID_ARG;  // K=V caches only
+  if (include_new != 0 && include_new != 1) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (!partial_o || !partial_lse || !q_pos_offset) return GEMMA_ATTN_ERR_INVALID_ARG;
+  if (include_new && !new_k) return GEMMA_ATTN_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  // without new keys the kernels never read new_k: q stands in for the pointer checks
+  const int rc = decode_prepare(params, q, include_new ? new_k : q, nullptr, k_cache, nullptr,
+                                GEMMA_ATTN_CACHE_CONTIGUOUS, cache_capacity, shard_seqlens, batch, n_q,
+                                max_shard_len, num_splits, &a);
+  if (rc != GEMMA_ATTN_OK) return rc;
+  if (reinterpret_cast<uintptr_t>(q_pos_offset) & 3u) return GEMMA_ATTN_ERR_MISALIGNED;
+  a.q_pos_offset = q_pos_offset;
+  a.new_keys = include_new;
+  if (!include_new) a.new_k = nullptr;
   a.partial_o = partial_o; a.partial_lse = partial_lse;
   if (launch_decode(a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) return GEMMA_ATTN_ERR_LAUNCH;
   t_launches = 1;

@@ -129,7 +129,8 @@ decode_tc_kernel(DecodeArgs a) {
   const bool kv_same = a.v_cache == nullptr;
   const int len = a.cache_seqlens[b];
   const int first = a.is_local ? max(0, len - a.window + 1) : 0;  // oldest position any query sees
-  const int nk = (len - first) + a.n_q;
+  const int nk = (len - first) + (a.new_keys ? a.n_q : 0);
+  const int qoff = a.q_pos_offset ? a.q_pos_offset[b] : 0;  // queries after a key-range shard
   const int per = (nk + a.num_splits - 1) / a.num_splits;
   const int v_lo = min(nk, split * per);
   const int v_hi = min(nk, v_lo + per);
@@ -187,7 +188,7 @@ decode_tc_kernel(DecodeArgs a) {
       y0 = x0; y1 = x1;
       if (j < r) {
         float c, s;
-        rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
+        rope_cos_sin((double)(len + i + qoff), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
         y0 = x0 * c - x1 * s;
         y1 = x0 * s + x1 * c;
       }
@@ -373,7 +374,7 @@ decode_tc_kernel(DecodeArgs a) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int row = nt * 8 + 2 * t + e;
-        const int qpos = len + (row < R ? row / group : 0);
+        const int qpos = len + qoff + (row < R ? row / group : 0);
         float mx = -INFINITY;
 #pragma unroll
         for (int hk = 0; hk < 2; ++hk) {
@@ -616,7 +617,8 @@ decode_warp_kernel(DecodeArgs a) {
   const bool kv_same = a.v_cache == nullptr;
   const int len = a.cache_seqlens[b];
   const int first = a.is_local ? max(0, len - a.window + 1) : 0;  // oldest position any query sees
-  const int nk = (len - first) + a.n_q;
+  const int nk = (len - first) + (a.new_keys ? a.n_q : 0);
+  const int qoff = a.q_pos_offset ? a.q_pos_offset[b] : 0;  // queries after a key-range shard
   const int per = (nk + a.num_splits - 1) / a.num_splits;
   const int v_lo = min(nk, split * per);
   const int v_hi = min(nk, v_lo + per);
@@ -739,7 +741,7 @@ decode_warp_kernel(DecodeArgs a) {
     const int i = row / group;
     const float x0 = bf2f(qs[row * KST + j]), x1 = bf2f(qs[row * KST + j + HALF]);
     float c, s;
-    rope_cos_sin((double)(len + i), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
+    rope_cos_sin((double)(len + i + qoff), rope_inv_freq_turns(j, D, a.log2_base), &c, &s);
     qs[row * KST + j] = f2bf(x0 * c - x1 * s);
     qs[row * KST + j + HALF] = f2bf(x0 * s + x1 * c);
   }
@@ -770,7 +772,7 @@ decode_warp_kernel(DecodeArgs a) {
   for (int e = 0; e < 2; ++e) {
     const int row = 2 * t + e;
     row_ok[e] = row < R;
-    qpos[e] = len + (row < R ? row / group : 0);
+    qpos[e] = len + qoff + (row < R ? row / group : 0);
   }
   const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
@@ -1124,6 +1126,7 @@ bool decode_supported(const DecodeArgs& a) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  if (decode_umma_applies(a)) return launch_decode_umma_any(a, stream);
   switch (a.head_dim) {
     case 32: return launch_decode_d<32>(a, stream);
     case 64: return launch_decode_d<64>(a, stream);

@@ -87,8 +87,20 @@ struct DecodeArgs {
   int r;
   double log2_base;
   float softmax_scale;
+  // A key-range shard of a longer history (global layers): the queries sit q_pos_offset[b]
+  // positions later than the shard's own end, and new_keys = 0 leaves the n_q new tokens out
+  // of the keys (another shard holds them). Defaults: no offset, new_keys = 1.
+  const int32_t* q_pos_offset;
+  int new_keys;
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Global (K=V, contiguous cache) layers with 9-32 query rows per KV head at head dim 256 or
+// 512 and at most 64 rotated pairs: the tcgen05 verify kernel (decode_umma.cu).
+bool decode_umma_applies(const DecodeArgs& a);
+cudaError_t launch_decode_umma_any(const DecodeArgs& a, cudaStream_t stream);
+// 3-D bf16 tensor map over a decode cache [planes][capacity][d] with {64, 128, 1} boxes,
+// 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* m, const void* base, int d, int capacity, int planes);
 int decode_max_rows(int head_dim);  // largest group * n_q one decode CTA handles
 bool decode_supported(const DecodeArgs& a);  // a kernel variant fits this shape
 

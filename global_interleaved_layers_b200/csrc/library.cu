@@ -4,6 +4,7 @@
 #include "rope.cu"
 #include "prefill.cu"
 #include "decode.cu"
+#include "decode_umma.cu"
 #include "decode_noalloc.cu"
 #include "append.cu"
 #include "selftest.cu"

@@ -125,6 +125,8 @@ def test_prefill_tiny_config_both_layers():
     (W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.0, rope_base=1e6), (300,)),
     (W.LayerSpec(W.GLOBAL, 8, 1, 256, rope_p=0.25, rope_base=1e4), (390,)),
     (W.LayerSpec(W.GLOBAL, 8, 1, 64, rope_p=0.25, rope_base=1e4), (260,)),
+    (W.LayerSpec(W.LOCAL, 4, 2, 512, window=150, rope_p=0.25, rope_base=1e4), (333, 64)),
+    (W.LayerSpec(W.GLOBAL, 4, 2, 512, rope_p=1.0, rope_base=1e4), (129, 65)),
 ])
 def test_prefill_shapes(layer, lens):
     _check_prefill(layer, lens, seed=3)
@@ -227,7 +229,7 @@ def _rotated_history(k_hist_b, n, layer):
     return out
 
 
-def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11, keys_rotated=False):
+def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11, keys_rotated=False, junk=False):
     B = len(cache_lens)
     Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
     rng_seed = seed
@@ -246,9 +248,13 @@ def _check_decode(layer, cache_lens, n_q, layout, num_splits=None, seed=11, keys
         kc = np.stack([ring_from_history(k_cache_src[b][:cache_lens[b]], cap) for b in range(B)])
         vc = None if layer.k_eq_v else np.stack([ring_from_history(v_hist[b][:cache_lens[b]], cap) for b in range(B)])
     else:
-        cap = max(max_len, 1)
+        cap = max(max_len, 1) + (200 if junk else 0)
         kc = np.zeros((B, Hkv, cap, d), np.uint16)
         vc = None if layer.k_eq_v else np.zeros((B, Hkv, cap, d), np.uint16)
+        if junk:  # rows past each sequence's cached tokens hold NaNs: the kernels must not read them
+            kc[:] = 0x7FC0
+            if vc is not None:
+                vc[:] = 0x7FC0
         for b, n in enumerate(cache_lens):
             kc[b, :, :n] = k_cache_src[b][:n].transpose(1, 0, 2)
             if vc is not None:
@@ -377,3 +383,25 @@ def test_prefill_divergent_rescale_within_warp():
     ref, ref_lse = oracle.attention(layer.kind, 0, 0.0, 1e4, layer.softmax_scale, q, k, None, pos, cu)
     assert_close(out.cpu().numpy(), ref, "divergent rescale")
     np.testing.assert_allclose(lse.cpu().numpy().T, ref_lse, atol=1e-2, rtol=0)
+
+
+# 9-32 query rows per KV head of a global layer (the speculative verify of 4 draft tokens
+# with 8 query heads per KV head is 32): the tcgen05 kernel (keys on M, rows on N), and with
+# GEMMA_ATTN_DECODE_MMA_SYNC=1 the mma.sync kernel, against the oracle. Cache rows past each
+# sequence's tokens hold NaNs; lengths straddle the 128-key tiles.
+GLO8 = W.LayerSpec(W.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
+
+
+@pytest.mark.parametrize("mma_sync", [False, True])
+@pytest.mark.parametrize("layer,cache_lens,n_q,splits", [
+    (GLO8, (0, 1, 127, 128, 129, 1000), 4, None),
+    (GLO8, (255, 256, 3000), 4, 3),
+    (GLO8, (700, 40), 2, 1),
+    (W.LayerSpec(W.GLOBAL, 16, 2, 512, rope_p=0.0, rope_base=1e6), (300, 129), 3, 2),
+    (W.LayerSpec(W.GLOBAL, 8, 1, 256, rope_p=0.25, rope_base=1e4), (500, 64), 4, 2),
+    (W.LayerSpec(W.GLOBAL, 4, 1, 512, rope_p=0.125, rope_base=1e6), (333,), 3, 1),
+])
+def test_decode_verify_rows_kernels(layer, cache_lens, n_q, splits, mma_sync, monkeypatch):
+    if mma_sync:
+        monkeypatch.setenv("GEMMA_ATTN_DECODE_MMA_SYNC", "1")
+    _check_decode(layer, cache_lens, n_q, G.CACHE_CONTIGUOUS, splits, seed=13, junk=True)
