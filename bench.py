@@ -563,6 +563,8 @@ def main():
         if not args.no_decode:
             per_kind.update(bench_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks,
                                          barrier))
+            per_kind["sharded_global_decode_256k"] = bench_sharded_decode(G, torch, dev, stream, flush_l2, peaks,
+                                                                          args, world, max_over_ranks, barrier)
         per_kind["vision_bidir_prefill"] = bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world,
                                                         max_over_ranks, barrier)
 
@@ -869,6 +871,65 @@ def bench_decode_workload(G, torch, dev, stream, flush_l2, peaks, args, max_over
             "note": "one launch per decode step; launch-bound (the rows are a few hundred KB)"}
         del kc, vc
         torch.cuda.empty_cache()
+
+
+def bench_sharded_decode(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):
+    """One decode step of a global layer over 8 sequences of 262,144 cached tokens (the 256K
+    context), the history split over the job's ranks by key range: each rank decodes its
+    range, the fp32 partials are all-gathered (NCCL) and combined on every rank. With one
+    rank this is the plain decode over the whole context."""
+    from global_interleaved_layers_b200.sharded import ShardedDecode, query_offsets
+    layer = W.LayerSpec(W.GLOBAL, 32, 4, 512, rope_p=0.25, rope_base=1e6)
+    B, n_q, L = 8, 1, 262144
+    Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
+    rank = int(os.environ.get("RANK", "0"))
+    offs = query_offsets([L] * B, world, rank)
+    shard = max(o[1] for o in offs)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(55 + rank)
+    kc = torch.empty((B, Hkv, max(shard, 1), d), dtype=torch.bfloat16, device=dev).normal_(generator=gen)
+    q = torch.randn((B, n_q, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    nk = torch.randn((B, n_q, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    lens = torch.tensor([o[1] for o in offs], dtype=torch.int32, device=dev)
+    qoff = torch.tensor([o[2] for o in offs], dtype=torch.int32, device=dev)
+    p = G.params(layer.kind, Hq, Hkv, d, rope_p=layer.rope_p, rope_base=layer.rope_base,
+                 softmax_scale=layer.softmax_scale)
+    splits = G.gemma_attn_decode_num_splits(p, B, n_q, shard)
+    dec = ShardedDecode(p, B, n_q, splits, dev)
+    out = torch.empty((B, n_q, Hq, d), dtype=torch.bfloat16, device=dev)
+
+    def one():
+        dec(q, nk, kc, kc.shape[2], lens, qoff, shard, out, None, stream)
+
+    log("sharded decode")
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    barrier()
+    evs = []
+    for _ in range(args.steps):
+        flush_l2()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    G.gemma_attn_check()
+    barrier()
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+    total_bytes = W.decode_cache_bytes(B, [L] * B, layer)  # every rank's range, read once
+    gbs = total_bytes / (ms * 1e-3) / 1e9
+    res = {"gbs": gbs, "ms": ms, "bytes": total_bytes, "ranks": world, "splits_per_rank": splits,
+           "frac_of_hbm_per_gpu": gbs / world / peaks["hbm_gbs"],
+           "gathered_bytes_per_rank": splits * B * n_q * Hq * (d + 1) * 4 * world,
+           "shape": f"B={B} n_q={n_q} Hq={Hq} Hkv={Hkv} d={d}, {L} cached tokens per sequence, "
+                    f"split by key range over {world} rank(s); decode + all-gather + combine"}
+    del kc, dec
+    torch.cuda.empty_cache()
+    return res
 
 
 def bench_vision(G, torch, dev, stream, flush_l2, peaks, args, world, max_over_ranks, barrier):

@@ -73,13 +73,14 @@ _lib.gemma_attn_combine.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_tile_plan.argtypes = [_I, _I, _P, _I, _I, _I, _P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
 _lib.gemma_attn_decode_noalloc.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.gemma_attn_cache_append.argtypes = [_PP, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P]
+_lib.gemma_attn_decode_shard.argtypes = [_PP, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P]
 _lib.gemma_attn_check.argtypes = [_P]
 _lib.gemma_attn_selftest_umma.argtypes = [_I, _P, _P, _P, _P, _P]
 _lib.gemma_attn_selftest_timeout.argtypes = [_P, _P]
 for _f in ("gemma_attn_prefill_workspace_size", "gemma_attn_prefill", "gemma_attn_decode",
            "gemma_attn_decode_num_splits", "gemma_attn_combine", "gemma_attn_tile_plan", "gemma_attn_check",
            "gemma_attn_selftest_umma", "gemma_attn_decode_noalloc", "gemma_attn_selftest_timeout",
-           "gemma_attn_cache_append",
+           "gemma_attn_cache_append", "gemma_attn_decode_shard",
            "gemma_attn_prefill_rotate", "gemma_attn_prefill_attend"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -169,6 +170,16 @@ def gemma_attn_decode(p: GemmaAttnParams, q, new_k, new_v, k_cache, v_cache, cac
                                   _ptr(v_cache), cache_layout, cache_capacity, _ptr(cache_seqlens), batch, n_q,
                                   max_cache_len, _ptr(partial_o), _ptr(partial_lse), num_splits, _stream(stream)),
            "gemma_attn_decode")
+
+
+def gemma_attn_decode_shard(p: GemmaAttnParams, q, new_k, k_cache, cache_capacity: int, shard_seqlens,
+                            q_pos_offset, include_new: bool, batch: int, n_q: int, max_shard_len: int, partial_o,
+                            partial_lse, num_splits: int, stream=None) -> None:
+    """Split-KV partials over one key-range shard of a longer K=V history (global layers)."""
+    _check(_lib.gemma_attn_decode_shard(ctypes.byref(p), _ptr(q), _ptr(new_k), _ptr(k_cache), cache_capacity,
+                                        _ptr(shard_seqlens), _ptr(q_pos_offset), 1 if include_new else 0, batch,
+                                        n_q, max_shard_len, _ptr(partial_o), _ptr(partial_lse), num_splits,
+                                        _stream(stream)), "gemma_attn_decode_shard")
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

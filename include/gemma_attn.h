@@ -250,6 +250,34 @@ int gemma_attn_cache_append(const gemma_attn_params* params, const void* new_k, 
                             void* k_cache, void* v_cache, int32_t cache_layout, int32_t cache_capacity,
                             const int32_t* cache_seqlens, int32_t batch, int32_t n_q, void* stream);
 
+/*
+ * Decode / verify over one key-range shard of a long K=V history (GLOBAL layers only), for
+ * a history spread over several GPUs: each GPU holds a contiguous range of every sequence's
+ * tokens and runs this on its range; the fp32 partials of all GPUs, stacked as splits
+ * (GPU-major), go through gemma_attn_combine (in-memory on one GPU, or after an all-gather
+ * between GPUs) to give the attention over the whole history. The medium models' 256K
+ * context is what makes one GPU's cache too small ("Visão geral do modelo Gemma 4", section
+ * "Recursos": the context window); the scores are those of the whole history because a rotation depends only
+ * on the distance between the query and the key ("Visual guide to Gemma 4", section
+ * "p-RoPE").
+ *   Arguments: q, new_k as gemma_attn_decode (new_k may be NULL when include_new is 0);
+ *   k_cache [batch, num_kv_heads, cache_capacity, head_dim] bf16 holding the shard's tokens
+ *   at rows 0 .. shard_seqlens[b] - 1 (device int32 [batch]); q_pos_offset (device int32
+ *   [batch], 4-byte aligned): how many tokens of sequence b come after the shard and before
+ *   the new tokens, i.e. the queries sit at shard-local positions shard_seqlens[b] +
+ *   q_pos_offset[b] + i; include_new: 1 for the shard that ends the history (its offset
+ *   must be 0), whose keys then also include the n_q new tokens (causally), 0 for the
+ *   others; max_shard_len >= every shard_seqlens[b]; partial_o / partial_lse / num_splits as
+ *   gemma_attn_decode (an empty shard writes lse = -inf, which the combine skips).
+ *   Errors: GEMMA_ATTN_ERR_INVALID_ARG for a LOCAL or BIDIR kind or a bad flag, otherwise
+ *   as gemma_attn_decode.
+ */
+int gemma_attn_decode_shard(const gemma_attn_params* params, const void* q, const void* new_k,
+                            const void* k_cache, int32_t cache_capacity, const int32_t* shard_seqlens,
+                            const int32_t* q_pos_offset, int32_t include_new, int32_t batch, int32_t n_q,
+                            int32_t max_shard_len, float* partial_o, float* partial_lse,
+                            int32_t num_splits, void* stream);
+
 /* A split count for gemma_attn_decode that fills the GPU for this shape. */
 int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,
                                  int32_t max_cache_len, int32_t* num_splits);

@@ -203,3 +203,19 @@ def test_decode_split_hint():
     assert s >= 1 and 8 * 4 * s >= 148
     loc = _p(num_q_heads=32, num_kv_heads=16, window=1024)
     assert G.gemma_attn_decode_num_splits(loc, 8, 1, 5) == 1
+
+
+def test_shard_entry_point_argument_rules():
+    # rejected before any launch: no device is needed
+    loc = G.params(G.LOCAL, 8, 4, 256, window=64)
+    glo = G.params(G.GLOBAL, 8, 1, 512, rope_p=0.25, rope_base=1e6)
+    fake = 1 << 20
+    with pytest.raises(G.GemmaAttnError) as e:  # local layers hold only a window: no shards
+        G.gemma_attn_decode_shard(loc, fake, fake, fake, 64, fake, fake, True, 1, 1, 64, fake, fake, 1)
+    assert e.value.status == G.ERR_INVALID_ARG
+    with pytest.raises(G.GemmaAttnError) as e:  # the shard that ends the history needs the new keys
+        G.gemma_attn_decode_shard(glo, fake, None, fake, 64, fake, fake, True, 1, 1, 64, fake, fake, 1)
+    assert e.value.status == G.ERR_INVALID_ARG
+    with pytest.raises(G.GemmaAttnError) as e:  # no offsets
+        G.gemma_attn_decode_shard(glo, fake, None, fake, 64, fake, None, False, 1, 1, 64, fake, fake, 1)
+    assert e.value.status == G.ERR_INVALID_ARG
