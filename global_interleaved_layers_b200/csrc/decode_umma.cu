@@ -17,7 +17,7 @@
 // place in the key ring; the value ring keeps them as stored.
 //
 // Roles (512 threads):
-//   warp 0      key-ring producer: TMA loads, chunk by chunk (the rotated chunks first)
+//   warp 0      key-ring producer: TMA loads, chunk by chunk (the rotated chunks last)
 //   warp 1      TMEM owner and issuer of the score MMAs, which run ahead into the next
 //               tile (its scores overlap this tile's softmax)
 //   warp 2      value-ring producer
@@ -77,11 +77,14 @@ struct __align__(8) UmmaHeader {
 };
 static_assert(sizeof(UmmaHeader) <= kUHeaderBytes, "header");
 
-// Chunk order of a key tile in the key ring: the two rotated chunks first.
+// Chunk order of a key tile in the key ring: the chunks without rotated dims first, the two
+// rotated ones (0 and d/128) last, so the ring keeps streaming while they are turned.
 template <int D>
 __device__ __forceinline__ int key_chunk(int i) {
-  constexpr int R = D / 128;
-  return i == 0 ? 0 : (i == 1 ? R : (i <= R ? i - 1 : i));
+  constexpr int kCh = D / 64, R = D / 128;
+  if (i == kCh - 2) return 0;
+  if (i == kCh - 1) return R;
+  return i + 1 + (i + 1 >= R ? 1 : 0);
 }
 
 }  // namespace
@@ -250,7 +253,7 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
             const int c = key_chunk<D>(i);
             const int s = kseq % kUKSlots;
             ok = mbar_wait(&hd->k_full[s], (uint32_t)(kseq / kUKSlots) & 1u, abort_flag);
-            if (ok && i == 0) ok = mbar_wait(&hd->rot_ready[lt & 1], (uint32_t)(lt >> 1) & 1u, abort_flag);
+            if (ok && i == kCh - 2) ok = mbar_wait(&hd->rot_ready[lt & 1], (uint32_t)(lt >> 1) & 1u, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const uint64_t kd = sdesc_sw128(smem_u32(kring + s * kUChunkBytes), 16, 1024);
@@ -305,16 +308,25 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
     bool ok = true;
     for (int lt = 0; lt < nt && ok; ++lt) {
       const int key0 = (t0 + lt) * kUKeys;
-      const int sq0 = lt * kCh;  // key-ring sequence index of the tile's chunk 0; chunk d/128 follows
+      const int sq0 = lt * kCh + kCh - 2;  // key-ring sequence index of the tile's chunk 0; chunk d/128 follows
       const int s0 = sq0 % kUKSlots, s1 = (sq0 + 1) % kUKSlots;
-      // A parity wait is only exact while the slot's previous fill has completed: those
-      // fills belong to tile t-1, whose score MMA has consumed them once S^T(t-1) is done.
+      // A parity wait is exact only while the slot's previous fill has completed and the next
+      // cannot have: the next needs this rotation. Fills of tile t-1 have completed once
+      // S^T(t-1) is done; a previous fill within this tile (sequence index minus the slot
+      // count) has once the score MMA released it (its release cannot advance again before
+      // this rotation either).
       if (lt >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(&hd->s_full[(lt - 1) & 1], (uint32_t)((lt - 1) >> 1) & 1u, abort_flag));
         if (!ok) break;
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&hd->k_full[s0], (uint32_t)(sq0 / kUKSlots) & 1u, abort_flag));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&hd->k_full[s1], (uint32_t)((sq0 + 1) / kUKSlots) & 1u, abort_flag));
+#pragma unroll
+      for (int e = 0; e < 2 && ok; ++e) {
+        const int sq = sq0 + e;
+        if (sq - kUKSlots >= lt * kCh)
+          ok = __all_sync(0xffffffffu, mbar_wait(&hd->k_empty[(sq - kUKSlots) % kUKSlots],
+                                                 (uint32_t)((sq - kUKSlots) / kUKSlots) & 1u, abort_flag));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&hd->k_full[sq % kUKSlots], (uint32_t)(sq / kUKSlots) & 1u, abort_flag));
+      }
       if (!ok) break;
       uint8_t* c0 = kring + s0 * kUChunkBytes;
       uint8_t* c1 = kring + s1 * kUChunkBytes;
