@@ -39,10 +39,11 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 # DRAM bytes (read + write) per launch of the global layer's attention kernel on the
-# headline block, from an ncu capture (see the profile summaries). Reported only while the
-# kernel's sources (their code: comments and blank lines do not count) still hash to the
-# captured state; any change makes it null until re-captured.
-NCU_TRAFFIC = {"bytes": None, "sources_sha256_16": "",
+# headline block: an ncu capture of the same sequence length with a quarter of the heads
+# (8 query heads, 1 KV head), scaled by 4 (the work units and their bytes scale with the
+# heads). Reported only while the kernel's sources (their code: comments and blank lines do
+# not count) still hash to the captured state; any change makes it null until re-captured.
+NCU_TRAFFIC = {"bytes": 4 * (334923776 + 233282048), "sources_sha256_16": "661f32af2124420b",
                "sources": ["global_interleaved_layers_b200/csrc/prefill.cu",
                            "global_interleaved_layers_b200/csrc/common.cuh",
                            "global_interleaved_layers_b200/csrc/tile_plan.h",
@@ -445,8 +446,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="only the headline block (no per_kind extras)")
     ap.add_argument("--case", default="block",
-                    choices=["block", "global_prefill", "local_prefill", "global_prefill_31b_h8",
-                             "global_decode", "local_decode", "global_verify"],
+                    choices=["block", "global_prefill", "local_prefill", "global_prefill_31b_h8", "local_prefill_31b",
+                             "global_decode", "local_decode", "global_verify", "vision_prefill"],
                     help="block: the benchmark (one JSON line). Any other value runs only that operation "
                          "(warmup + steps launches, no timing contract) for profiler captures.")
     ap.add_argument("--ctx", type=int, default=0, help="decode cases: cached tokens per sequence (0: 131072)")
@@ -991,9 +992,31 @@ def run_case(args):
     stream = torch.cuda.current_stream()
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
-    if "prefill" in args.case:
+    if args.case == "vision_prefill":
+        wl = W.vision_batch()
+        layer = wl.layers[0]
+        T = wl.total_tokens
+        q = torch.randn((T, layer.num_q_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        k = torch.randn((T, layer.num_kv_heads, layer.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+        v = torch.randn_like(k)
+        out = torch.empty_like(q)
+        idx = np.concatenate([np.arange(n) for n in wl.seq_lens])
+        hw = torch.from_numpy(np.stack([idx // 56, idx % 56], axis=1).astype(np.int32)).to(dev)
+        cu = torch.from_numpy(wl.cu_seqlens()).to(dev)
+        p = G.params(layer.kind, layer.num_q_heads, layer.num_kv_heads, layer.head_dim, rope_p=1.0,
+                     rope_base=layer.rope_base, softmax_scale=layer.softmax_scale)
+        ws_bytes = G.gemma_attn_prefill_workspace_size(p, T)
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+        def op():
+            G.gemma_attn_prefill(p, q, k, v, out, None, hw, cu, len(wl.seq_lens), T, max(wl.seq_lens), ws, ws_bytes,
+                                 stream)
+    elif "prefill" in args.case:
         wl = W.e2b_block()
         layer = wl.layers[-1] if args.case == "global_prefill" else wl.layers[0]
+        if args.case == "local_prefill_31b":
+            wl = W.b31_block()
+            layer = wl.layers[0]
         if args.case == "global_prefill_31b_h8":
             # the 31B global layer's sequence length with a quarter of its heads (8 query heads,
             # one KV head): DRAM traffic per launch scales with the heads, for a capture that
