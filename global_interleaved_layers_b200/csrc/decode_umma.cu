@@ -27,10 +27,11 @@
 //               taking rows 0-15 and the other rows 16-31; row maxima and sums reduced
 //               across the lanes and the four warps of a row half; P^T into shared memory
 //               (double-buffered); output rescale; epilogue O / l and log-sum-exp
-// The last tile of a sequence (cached rows, then the new tokens, then zeros) is assembled
-// by the producer warps with plain copies instead of TMA: rows past the cache hold no data
-// the kernel may read. Every wait is bounded: one that runs out records a timeout and the
-// CTA unwinds.
+// The last tile of a sequence (cached rows, then the new tokens, then zeros) is loaded by
+// TMA like any other and then patched by the producer warp: the rows past the cache end
+// hold no data the kernel may use, so they are overwritten in shared memory with the new
+// tokens' rows and zeros before the chunk is released to its consumers. Every wait is
+// bounded: one that runs out records a timeout and the CTA unwinds.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -61,6 +62,7 @@ __device__ __forceinline__ uint32_t sw128(int row, int colb) {
 struct __align__(8) UmmaHeader {
   uint64_t k_full[kUKSlots], k_empty[kUKSlots];
   uint64_t v_full[kUVSlots], v_empty[kUVSlots];
+  uint64_t k_tail[kUKSlots], v_tail[kUVSlots];  // a tail chunk's TMA landed (before the patch)
   uint64_t q_ready;     // softmax warps: the query rows are in shared memory
   uint64_t rot_ready[2];  // rotation warps: tile t's rotated chunks are in place (barrier t & 1)
   uint64_t s_full[2];   // S^T(t) complete (buffer t & 1)
@@ -140,6 +142,8 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUKSlots; ++s) { mbar_init(&hd->k_full[s], 1); mbar_init(&hd->k_empty[s], 1); }
     for (int s = 0; s < kUVSlots; ++s) { mbar_init(&hd->v_full[s], 1); mbar_init(&hd->v_empty[s], 1); }
+    for (int s = 0; s < kUKSlots; ++s) mbar_init(&hd->k_tail[s], 1);
+    for (int s = 0; s < kUVSlots; ++s) mbar_init(&hd->v_tail[s], 1);
     mbar_init(&hd->q_ready, 8);
     mbar_init(&hd->rot_ready[0], 4);
     mbar_init(&hd->rot_ready[1], 4);
@@ -174,17 +178,17 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
   const uint32_t col_o = 64;
   volatile int* abort_flag = &hd->abort_flag;
 
-  // The sequence's last tile (it holds keys at or past the cache end) is assembled with
-  // plain copies by the whole producer warp: cached rows, then the new tokens, then zeros.
-  auto copy_tail_chunk = [&](uint8_t* dst, int c, int key0) {
-    for (int idx = lane; idx < kUKeys * 8; idx += 32) {
+  // A tile that reaches past the cache end (the sequence's last one or two) is patched by
+  // the whole producer warp once its TMA load (if any) has landed: rows from the cache end
+  // on take the new tokens' rows, then zeros (finite values: the value product multiplies
+  // them by zero weights).
+  auto patch_tail_chunk = [&](uint8_t* dst, int c, int key0) {
+    const int u0 = len - key0 > 0 ? len - key0 : 0;  // first row past the cache
+    for (int idx = u0 * 8 + lane; idx < kUKeys * 8; idx += 32) {
       const int u = idx >> 3, k16 = idx & 7;
       const int v = key0 + u;
       uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (v < len)
-        val = *reinterpret_cast<const uint4*>(a.k_cache + (((size_t)b * a.num_kv_heads + kvh) * a.capacity + v) * D +
-                                               c * 64 + k16 * 8);
-      else if (v < nk)
+      if (v < nk)
         val = *reinterpret_cast<const uint4*>(a.new_k + (((size_t)b * a.n_q + (v - len)) * a.num_kv_heads + kvh) * D +
                                                c * 64 + k16 * 8);
       *reinterpret_cast<uint4*>(dst + sw128(u, k16 * 16)) = val;
@@ -199,11 +203,26 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
     const int nslots = is_k ? kUKSlots : kUVSlots;
     uint64_t* full = is_k ? hd->k_full : hd->v_full;
     uint64_t* empty = is_k ? hd->k_empty : hd->v_empty;
+    uint64_t* tailb = is_k ? hd->k_tail : hd->v_tail;
     uint8_t* ring = is_k ? kring : vring;
     if (lane == 0 && nt > 0) prefetch_tensormap(&cache_map);
     const int plane = b * a.num_kv_heads + kvh;
     bool ok = true;
     int seq = 0;
+    // A tail chunk whose cache rows are on their way: it is patched and released one
+    // chunk later, so its load overlaps the next chunk's (slot s, parity bit per slot).
+    int pend_s = -1, pend_c = 0, pend_key0 = 0;
+    uint32_t tail_par = 0u;
+    auto finish_pending = [&]() -> bool {
+      if (pend_s < 0) return true;
+      const int s = pend_s;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tailb[s], (tail_par >> s) & 1u, abort_flag))) return false;
+      pend_s = -1;
+      tail_par ^= 1u << s;
+      patch_tail_chunk(ring + s * kUChunkBytes, pend_c, pend_key0);
+      if (lane == 0) mbar_arrive(&full[s]);
+      return true;
+    };
     for (int lt = 0; lt < nt && ok; ++lt) {
       const int key0 = (t0 + lt) * kUKeys;
       const bool tail = key0 + kUKeys > len;
@@ -218,11 +237,34 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
             mbar_arrive_expect_tx(&full[s], kUChunkBytes);
             tma_load_3d(dst, &cache_map, &full[s], c * 64, key0, plane);
           }
-        } else {
-          copy_tail_chunk(dst, c, key0);
-          if (lane == 0) mbar_arrive(&full[s]);
+        } else if (key0 < len) {  // cache rows by TMA (rows past the capacity read as zeros)
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&tailb[s], kUChunkBytes);
+            tma_load_3d(dst, &cache_map, &tailb[s], c * 64, key0, plane);
+          }
+        }
+        // the previous chunk, if it was a tail chunk in flight: its slot was taken before
+        // this one, so the consumers see the chunks in order
+        ok = finish_pending();
+        if (!ok) break;
+        if (tail) {
+          if (key0 < len) {
+            pend_s = s; pend_c = c; pend_key0 = key0;
+          } else {  // no cached rows in this tile: new tokens and zeros only
+            patch_tail_chunk(dst, c, key0);
+            if (lane == 0) mbar_arrive(&full[s]);
+          }
         }
       }
+    }
+    if (ok) ok = finish_pending();
+    if (pend_s >= 0 && lane == 0) {
+      // an abort left a tail chunk's load in flight: it lands before the CTA can exit, and
+      // its slot is released so the drain below finds every fill complete
+      const uint32_t par = (tail_par >> pend_s) & 1u;
+      const unsigned long long ts = globaltimer_ns();
+      while (!mbar_try_wait(&tailb[pend_s], par) && globaltimer_ns() - ts < kWaitLimitNs) {}
+      mbar_arrive(&full[pend_s]);
     }
     // the last loads land before the CTA can exit (one per slot at most is outstanding)
     if (lane == 0) {
