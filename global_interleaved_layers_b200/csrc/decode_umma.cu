@@ -46,6 +46,7 @@ constexpr int kUChunkBytes = 16384;     // 128 keys x 64 dims bf16
 constexpr int kUKSlots = 6;             // key ring
 constexpr int kUVSlots = 4;             // value ring (chunk pairs stay adjacent)
 constexpr int kUHeaderBytes = 4096;     // mbarriers, TMEM base, flags, reductions, angle tables
+constexpr int kURankMax = 2048;         // sequences ranked by length in the P^T buffers (16 KB)
 
 __device__ __forceinline__ float ex2_sfu(float x) {
   float y;
@@ -72,7 +73,8 @@ struct __align__(8) UmmaHeader {
   uint64_t mma_done[2];  // each MMA issuer's last operations complete
   uint32_t tmem_base;
   int abort_flag;
-  int seq;              // the sequence this CTA serves
+  int seq;              // the sequence this CTA serves (-1: no work item)
+  int split, tile_per, seq_splits;  // its split, tiles per split, splits the sequence uses
   float red[2][2][4][16];  // [meeting parity][row half][quadrant][row]
   double itf[64];       // theta_j / (2 pi) of rotary pair j (0 past the rotated pairs)
   float2 stp[64];       // cos / sin of theta_j (identity past the rotated pairs)
@@ -99,9 +101,11 @@ constexpr size_t umma_smem_bytes() {
 
 template <int D>
 __global__ void __launch_bounds__(kUThreads, 1)
-decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) {
+decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, int num_sms) {
   constexpr int kCh = D / 64;        // chunks per key tile
   constexpr int kBlocks = D / 128;   // 128-dim blocks of O^T
+  static_assert(kCh * kUN * 128 >= kURankMax * 4 && 2 * kUN * 256 >= kURankMax * 8, "ranking tables");
+  static_assert(2 * kUN * 256 >= kUN * 64 * 8, "query angle table");
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   UmmaHeader* hd = reinterpret_cast<UmmaHeader*>(base);
@@ -110,30 +114,81 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
   uint8_t* kring = p_s + 2 * (size_t)kUN * 256;
   uint8_t* vring = kring + (size_t)kUKSlots * kUChunkBytes;
 
-  const int split = blockIdx.x, kvh = blockIdx.y;
+  const int kvh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // CTAs start in blockIdx order; blockIdx.z counts sequences from the longest down (ties by
-  // index), so the longest splits start first and the short ones fill the tail
-  if (threadIdx.x == 0) hd->seq = (int)blockIdx.z;
-  __syncthreads();
-  if (a.batch <= kUThreads && (int)threadIdx.x < a.batch) {
-    const int me = threadIdx.x, lme = a.cache_seqlens[me];
-    int rank = 0;
-    for (int o = 0; o < a.batch; ++o) {
-      const int lo = a.cache_seqlens[o];
-      rank += (lo > lme || (lo == lme && o < me)) ? 1 : 0;
+  // Work items. Every split of every sequence covers the same number of key tiles, T =
+  // max(the longest sequence's tiles / num_splits, all tiles / (4 waves of CTAs)), so the
+  // items are near-equal in work; a sequence uses ceil(tiles / T) of the num_splits splits.
+  // Items are numbered longest sequence first (ties by index), then by split, and CTA i of
+  // the KV head (blockIdx.x + num_splits * blockIdx.z) takes item i, so the longest work
+  // starts first and the short items fill the tail. CTAs past the last item leave at once;
+  // the last split of a sequence writes -inf log-sum-exps for the splits it leaves unused.
+  // (The lengths are staged in the Q^T buffer and the ranking table lives in the P^T
+  // buffers, both free until the query rows are loaded: one global load per length, not one
+  // dependent load per comparison.)
+  {
+    int* sl = reinterpret_cast<int*>(q_s);
+    int* rk_tiles = reinterpret_cast<int*>(p_s);
+    int* rk_seq = rk_tiles + kURankMax;
+    const int extra = a.new_keys ? a.n_q : 0;
+    if (a.batch <= kURankMax)
+      for (int i = threadIdx.x; i < a.batch; i += kUThreads) sl[i] = a.cache_seqlens[i];
+    __syncthreads();
+    if (a.batch <= kURankMax) {
+      for (int me = threadIdx.x; me < a.batch; me += kUThreads) {
+        const int lme = sl[me];
+        int rank = 0;
+        for (int o = 0; o < a.batch; ++o) {
+          const int lo = sl[o];
+          rank += (lo > lme || (lo == lme && o < me)) ? 1 : 0;
+        }
+        rk_tiles[rank] = (lme + extra + kUKeys - 1) / kUKeys;
+        rk_seq[rank] = me;
+      }
     }
-    if (rank == (int)blockIdx.z) hd->seq = me;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const bool ranked = a.batch <= kURankMax;
+      long long total = 0;
+      int mx = 0;
+      for (int r = 0; r < a.batch; ++r) {
+        const int tl = ranked ? rk_tiles[r] : (a.cache_seqlens[r] + extra + kUKeys - 1) / kUKeys;
+        total += tl;
+        mx = max(mx, tl);
+      }
+      total *= a.num_kv_heads;
+      const long long ctas = 4LL * (num_sms > 0 ? num_sms : 148);
+      int T = (int)((total + ctas - 1) / ctas);
+      T = max(T, (mx + a.num_splits - 1) / a.num_splits);
+      T = max(T, 1);
+      const int item = (int)blockIdx.x + a.num_splits * (int)blockIdx.z;
+      int acc = 0;
+      hd->seq = -1;
+      for (int r = 0; r < a.batch; ++r) {
+        const int tl = ranked ? rk_tiles[r] : (a.cache_seqlens[r] + extra + kUKeys - 1) / kUKeys;
+        const int sr = max(1, (tl + T - 1) / T);
+        if (item < acc + sr) {
+          hd->seq = ranked ? rk_seq[r] : r;
+          hd->split = item - acc;
+          hd->seq_splits = sr;
+          break;
+        }
+        acc += sr;
+      }
+      hd->tile_per = T;
+    }
+    __syncthreads();
   }
-  __syncthreads();
+  if (hd->seq < 0) return;  // no work item: nothing allocated or armed yet
   const int b = hd->seq;
+  const int split = hd->split;
   const int group = a.num_q_heads / a.num_kv_heads;
   const int R = group * a.n_q;
   const int len = a.cache_seqlens[b];
   const int nk = len + (a.new_keys ? a.n_q : 0);           // visible keys: the cache, then the new tokens
   const int qoff = a.q_pos_offset ? a.q_pos_offset[b] : 0;  // queries after a key-range shard
   const int ntiles = (nk + kUKeys - 1) / kUKeys;
-  const int per = (ntiles + a.num_splits - 1) / a.num_splits;
+  const int per = hd->tile_per;
   const int t0 = min(ntiles, split * per);
   const int nt = min(ntiles, t0 + per) - t0;
   const int rows_total = a.batch * a.n_q * a.num_q_heads;
@@ -352,6 +407,13 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
       const int key0 = (t0 + lt) * kUKeys;
       const int sq0 = lt * kCh + kCh - 2;  // key-ring sequence index of the tile's chunk 0; chunk d/128 follows
       const int s0 = sq0 % kUKSlots, s1 = (sq0 + 1) % kUKSlots;
+      // the anchors need no data: they are computed while the chunks are on their way
+      float ac[8], as[8];
+      {
+        const double pos0 = (double)(key0 + 8 * g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rope_cos_sin(pos0, hd->itf[8 * k + e], &ac[e], &as[e]);
+      }
       // A parity wait is exact only while the slot's previous fill has completed and the next
       // cannot have: the next needs this rotation. Fills of tile t-1 have completed once
       // S^T(t-1) is done; a previous fill within this tile (sequence index minus the slot
@@ -372,10 +434,6 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
       if (!ok) break;
       uint8_t* c0 = kring + s0 * kUChunkBytes;
       uint8_t* c1 = kring + s1 * kUChunkBytes;
-      float ac[8], as[8];
-      const double pos0 = (double)(key0 + 8 * g);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) rope_cos_sin(pos0, hd->itf[8 * k + e], &ac[e], &as[e]);
 #pragma unroll 2
       for (int i = 0; i < 8; ++i) {
         const uint32_t off = sw128(8 * g + i, 16 * k);
@@ -420,8 +478,11 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
 
     // ---- query rows, rotated for their positions, into the swizzled K-major layout: item
     // (row, unit ku) holds dims 8ku .. 8ku + 7 and their partners d/2 + 8ku ..; every thread
-    // issues all of its 16-byte loads before it computes
+    // issues all of its 16-byte loads before it computes. The angles depend only on the
+    // token and the pair: each is computed once into a table (in the P^T buffers, free
+    // until the first tile; n_q <= 32 tokens x r <= 64 pairs of cos / sin fill 16 KB at most).
     {
+      float2* qcs = reinterpret_cast<float2*>(p_s);
       constexpr int kU = D / 16;                  // 16-byte units in each half of a row
       constexpr int kItems = kUN * kU / 256;      // items per thread
       uint4 x0[kItems], x1[kItems];
@@ -435,6 +496,13 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
           x1[it] = *reinterpret_cast<const uint4*>(qrow + D / 2 + 8 * ku);
         }
       }
+      for (int idx = tid; idx < a.n_q * r; idx += 256) {
+        const int tok = idx / r, j = idx % r;
+        float cs, sn;
+        rope_cos_sin((double)(len + tok + qoff), hd->itf[j], &cs, &sn);
+        qcs[idx] = make_float2(cs, sn);
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the softmax warps' table is complete
 #pragma unroll
       for (int it = 0; it < kItems; ++it) {
         const int idx = tid + 256 * it, row = idx / kU, ku = idx % kU;
@@ -452,10 +520,9 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
             y0[e2] = a0;
             y1[e2] = a1;
             if (row < R && j < r) {
-              float cs, sn;
-              rope_cos_sin((double)(len + row / group + qoff), hd->itf[j], &cs, &sn);
-              y0[e2] = a0 * cs - a1 * sn;
-              y1[e2] = a0 * sn + a1 * cs;
+              const float2 t = qcs[(row / group) * r + j];
+              y0[e2] = a0 * t.x - a1 * t.y;
+              y1[e2] = a0 * t.y + a1 * t.x;
             }
           }
           y0w[h] = pack_bf16x2(y0[0], y0[1]);
@@ -629,8 +696,14 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a) 
         if (q < R) {
           const size_t orow = ((size_t)b * a.n_q + q / group) * a.num_q_heads + kvh * group + q % group;
           const float lse = (nt > 0 && lq > 0.f) ? (mq + log2f(lq)) * 0.6931471805599453f : -INFINITY;
-          if (a.out == nullptr) a.partial_lse[(size_t)split * rows_total + orow] = lse;
-          else if (a.out_lse != nullptr) a.out_lse[orow] = lse;
+          if (a.out == nullptr) {
+            a.partial_lse[(size_t)split * rows_total + orow] = lse;
+            const int seq_splits = hd->seq_splits;
+            if (split == seq_splits - 1)  // the sequence's splits past its last are empty
+              for (int sp = seq_splits; sp < a.num_splits; ++sp) a.partial_lse[(size_t)sp * rows_total + orow] = -INFINITY;
+          } else if (a.out_lse != nullptr) {
+            a.out_lse[orow] = lse;
+          }
         }
       }
     }
@@ -657,8 +730,11 @@ cudaError_t launch_decode_umma(const DecodeArgs& a, cudaStream_t stream) {
   }
   CUtensorMap map;
   if (!encode_cache_map(&map, a.k_cache, D, a.capacity, a.batch * a.num_kv_heads)) return cudaErrorInvalidValue;
+  static int sms_cached[64] = {0};
+  if (sms_cached[dev] == 0 && cudaDeviceGetAttribute(&sms_cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms_cached[dev] = 0;
   dim3 grid(a.num_splits, a.num_kv_heads, a.batch);
-  decode_umma_kernel<D><<<grid, kUThreads, smem, stream>>>(map, a);
+  decode_umma_kernel<D><<<grid, kUThreads, smem, stream>>>(map, a, sms_cached[dev]);
   return cudaGetLastError();
 }
 
