@@ -405,3 +405,17 @@ def test_decode_verify_rows_kernels(layer, cache_lens, n_q, splits, mma_sync, mo
     if mma_sync:
         monkeypatch.setenv("GEMMA_ATTN_DECODE_MMA_SYNC", "1")
     _check_decode(layer, cache_lens, n_q, G.CACHE_CONTIGUOUS, splits, seed=13, junk=True)
+
+
+@pytest.mark.parametrize("batch,splits", [(40, 5), (2060, 2)])
+def test_verify_work_items_over_ragged_batches(batch, splits):
+    """The tcgen05 verify kernel's work items (equal tile counts per split, longest sequence
+    first, unused splits left at -inf): a ragged batch with empty, one-tile and multi-tile
+    sequences, and a batch past the 2048 sequences the kernel ranks by length (those keep
+    their index order)."""
+    rng = np.random.default_rng(batch)
+    lens = rng.integers(0, 130, batch)
+    lens[:3] = (0, 1, 129)
+    if batch < 100:
+        lens[3:6] = (1500, 700, 2000)
+    _check_decode(GLO8, tuple(int(n) for n in lens), 4, G.CACHE_CONTIGUOUS, splits, seed=17, junk=batch < 100)
