@@ -2,9 +2,10 @@
 // tcgen05 tensor cores, for 9 to 32 query rows per KV head at head dim 256 or 512: the
 // 4-token verify of a draft model's tokens with 8 query heads per KV head is 32 rows.
 //
-// One CTA handles a (sequence, KV head, split): every query row of the KV head (the
-// group's heads x the new tokens) against a contiguous range of 128-key tiles of the
-// sequence's visible keys (the cached tokens, then the new tokens themselves). Keys sit on
+// One CTA handles a work item, a (sequence, KV head, split): every query row of the KV
+// head (the group's heads x the new tokens) against a contiguous range of 128-key tiles of
+// the sequence's visible keys (the cached tokens, then the new tokens themselves). Items
+// cover equal tile counts, so a long sequence takes more splits than a short one. Keys sit on
 // the MMA's M dimension, rows on N = 32:
 //   S^T = K Q^T     M = 128 keys, N = 32 rows, K = head dim (64-dim chunks)
 //   O^T += V^T P^T  M = 128 head dims per block (head_dim / 128 blocks), N = 32, K = 128 keys

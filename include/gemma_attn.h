@@ -176,7 +176,9 @@ int gemma_attn_prefill_attend(const gemma_attn_params* params, const void* q, co
  *   partial_o  [num_splits, batch * n_q * num_q_heads, head_dim] float32, written.
  *   partial_lse [num_splits, batch * n_q * num_q_heads] float32, written (-inf for an
  *              empty split). Row index = (b * n_q + i) * num_q_heads + h.
- *   The visible keys of each sequence are cut into num_splits contiguous ranges.
+ *   The visible keys of each sequence are cut into at most num_splits contiguous ranges,
+ *   in split order; a split with no keys (for a short sequence, the splits past its last)
+ *   has lse -inf and its partial_o row is not written (the combine does not read it).
  *   Limits: (num_q_heads / num_kv_heads) * n_q <= 64 (<= 32 for head_dim 512), else
  *   GEMMA_ATTN_ERR_UNSUPPORTED; q, new_k, new_v and the caches 16-byte aligned.
  */
