@@ -403,6 +403,16 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
     // pairs past r keep the identity (the tables hold cos 1, sin 0 for them)
     const int tid = threadIdx.x - 128;  // 0..127
     const int k = tid & 7, g = tid >> 3;
+    // this thread's pairs' frequencies and one-key steps, held in registers: read from
+    // shared memory inside the loop they would be reloaded after every store to the ring
+    // (and the lanes' stride of 8 pairs puts four lanes on each bank)
+    double itfv[8];
+    float2 stv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      itfv[e] = hd->itf[8 * k + e];
+      stv[e] = hd->stp[8 * k + e];
+    }
     bool ok = true;
     for (int lt = 0; lt < nt && ok; ++lt) {
       const int key0 = (t0 + lt) * kUKeys;
@@ -413,7 +423,7 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
       {
         const double pos0 = (double)(key0 + 8 * g);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) rope_cos_sin(pos0, hd->itf[8 * k + e], &ac[e], &as[e]);
+        for (int e = 0; e < 8; ++e) rope_cos_sin(pos0, itfv[e], &ac[e], &as[e]);
       }
       // A parity wait is exact only while the slot's previous fill has completed and the next
       // cannot have: the next needs this rotation. Fills of tile t-1 have completed once
@@ -452,7 +462,7 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
             const float x1 = __uint_as_float(e2 ? (x1w[h] & 0xFFFF0000u) : (x1w[h] << 16));
             y0[e2] = x0 * ac[e] - x1 * as[e];
             y1[e2] = x0 * as[e] + x1 * ac[e];
-            const float2 st = hd->stp[8 * k + e];
+            const float2 st = stv[e];
             const float nc = ac[e] * st.x - as[e] * st.y;
             as[e] = ac[e] * st.y + as[e] * st.x;
             ac[e] = nc;
