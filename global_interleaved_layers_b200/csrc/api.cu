@@ -381,6 +381,10 @@ int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch,
     const double cost = (double)waves * ((double)((keys + s - 1) / s) + kSplitOverheadKeys);
     if (s == 1 || cost < best_cost * (1.0 - 1e-9)) { best_cost = cost; best = s; }
   }
+  // The verify kernel picks its own tiles per split from the lengths it sees, among
+  // ceil(longest / s) for s up to the split count: twice the uniform choice leaves it room
+  // for ragged batches (no more than one split per 128-key tile).
+  if (decode_umma_shape(params, n_q)) best = std::max(1, std::min(2 * best, (keys + 127) / 128));
   *num_splits = best;
   return GEMMA_ATTN_OK;
 }

@@ -48,6 +48,7 @@ constexpr int kUKSlots = 6;             // key ring
 constexpr int kUVSlots = 4;             // value ring (chunk pairs stay adjacent)
 constexpr int kUHeaderBytes = 4096;     // mbarriers, TMEM base, flags, reductions, angle tables
 constexpr int kURankMax = 2048;         // sequences ranked by length in the P^T buffers (16 KB)
+constexpr int kUStartTiles = 3;         // a CTA's start-up cost, in 128-key tiles
 
 __device__ __forceinline__ float ex2_sfu(float x) {
   float y;
@@ -76,6 +77,9 @@ struct __align__(8) UmmaHeader {
   int abort_flag;
   int seq;              // the sequence this CTA serves (-1: no work item)
   int split, tile_per, seq_splits;  // its split, tiles per split, splits the sequence uses
+  int tile_floor, max_tiles, search;  // tile-count choice: 4-wave floor, longest sequence, on/off
+  long long cand_cost[16];  // estimated duration of each candidate tile count (one per warp)
+  int cand_tiles[16];
   float red[2][2][4][16];  // [meeting parity][row half][quadrant][row]
   double itf[64];       // theta_j / (2 pi) of rotary pair j (0 past the rotated pairs)
   float2 stp[64];       // cos / sin of theta_j (identity past the rotated pairs)
@@ -117,9 +121,11 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
 
   const int kvh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Work items. Every split of every sequence covers the same number of key tiles, T =
-  // max(the longest sequence's tiles / num_splits, all tiles / (4 waves of CTAs)), so the
-  // items are near-equal in work; a sequence uses ceil(tiles / T) of the num_splits splits.
+  // Work items. Every split of every sequence covers the same number of key tiles T, at
+  // least max(the longest sequence's tiles / num_splits, all tiles / (4 waves of CTAs)), so
+  // the items are near-equal in work; a sequence uses ceil(tiles / T) of the num_splits
+  // splits. T is the candidate ceil(longest / s), s <= num_splits, with the fewest rounds
+  // times tiles per round (below).
   // Items are numbered longest sequence first (ties by index), then by split, and CTA i of
   // the KV head (blockIdx.x + num_splits * blockIdx.z) takes item i, so the longest work
   // starts first and the short items fill the tail. CTAs past the last item leave at once;
@@ -148,8 +154,9 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
       }
     }
     __syncthreads();
+    const bool ranked = a.batch <= kURankMax;
+    const int sms = num_sms > 0 ? num_sms : 148;
     if (threadIdx.x == 0) {
-      const bool ranked = a.batch <= kURankMax;
       long long total = 0;
       int mx = 0;
       for (int r = 0; r < a.batch; ++r) {
@@ -158,10 +165,51 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
         mx = max(mx, tl);
       }
       total *= a.num_kv_heads;
-      const long long ctas = 4LL * (num_sms > 0 ? num_sms : 148);
-      int T = (int)((total + ctas - 1) / ctas);
-      T = max(T, (mx + a.num_splits - 1) / a.num_splits);
-      T = max(T, 1);
+      const long long ctas = 4LL * sms;
+      const int floor4 = max(1, (int)((total + ctas - 1) / ctas));
+      hd->tile_floor = floor4;
+      hd->max_tiles = mx;
+      hd->tile_per = max(floor4, (mx + a.num_splits - 1) / a.num_splits);
+      hd->search = ranked && a.num_splits > 1;
+    }
+    __syncthreads();
+    if (hd->search) {
+      // Candidates T = ceil(longest / s) for s = num_splits, num_splits - 1, ... (one per
+      // warp). A launch runs its items in rounds of one CTA per SM, and a round lasts about as
+      // long as its longest item, so a candidate costs (T + start-up) x ceil(items / SMs).
+      // Just more items than SMs makes a second round of long items; the fewest rounds of the
+      // shortest items win (ties to the larger T: fewer partials to combine).
+      const int w = threadIdx.x >> 5, ln = threadIdx.x & 31;
+      const int s_c = a.num_splits - w;
+      if (w < 16) {
+        long long cost = -1;
+        int Tc = 0;
+        if (s_c >= 1) {
+          Tc = max(hd->tile_floor, (hd->max_tiles + s_c - 1) / s_c);
+          int n = 0;
+          for (int r = ln; r < a.batch; r += 32) n += max(1, (rk_tiles[r] + Tc - 1) / Tc);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+          const long long items = (long long)n * a.num_kv_heads;
+          cost = (long long)(Tc + kUStartTiles) * ((items + sms - 1) / sms);
+        }
+        if (ln == 0) {
+          hd->cand_cost[w] = cost;
+          hd->cand_tiles[w] = Tc;
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        long long best = -1;
+        for (int c = 0; c < 16; ++c)
+          if (hd->cand_cost[c] >= 0 && (best < 0 || hd->cand_cost[c] <= best)) {
+            best = hd->cand_cost[c];
+            hd->tile_per = hd->cand_tiles[c];
+          }
+      }
+    }
+    if (threadIdx.x == 0) {
+      const int T = hd->tile_per;
       const int item = (int)blockIdx.x + a.num_splits * (int)blockIdx.z;
       int acc = 0;
       hd->seq = -1;
@@ -176,7 +224,6 @@ decode_umma_kernel(const __grid_constant__ CUtensorMap cache_map, DecodeArgs a, 
         }
         acc += sr;
       }
-      hd->tile_per = T;
     }
     __syncthreads();
   }
@@ -755,6 +802,15 @@ bool decode_umma_applies(const DecodeArgs& a) {
   if (e && e[0] == '1') return false;
   return a.v_cache == nullptr && !a.ring && !a.keys_rotated && (a.head_dim == 256 || a.head_dim == 512) && R > 8 &&
          R <= kUN && a.r <= 64 && (reinterpret_cast<uintptr_t>(a.k_cache) & 15u) == 0;
+}
+
+bool decode_umma_shape(const gemma_attn_params* p, int n_q) {
+  const char* e = getenv("GEMMA_ATTN_DECODE_MMA_SYNC");
+  if (e && e[0] == '1') return false;
+  if (p->kind != GEMMA_ATTN_GLOBAL || p->num_kv_heads < 1) return false;
+  const int R = (p->num_q_heads / p->num_kv_heads) * n_q;
+  return (p->head_dim == 256 || p->head_dim == 512) && R > 8 && R <= kUN &&
+         rotated_pairs(p->rope_p, p->head_dim) <= 64;
 }
 
 cudaError_t launch_decode_umma_any(const DecodeArgs& a, cudaStream_t stream) {

@@ -97,6 +97,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Global (K=V, contiguous cache) layers with 9-32 query rows per KV head at head dim 256 or
 // 512 and at most 64 rotated pairs: the tcgen05 verify kernel (decode_umma.cu).
 bool decode_umma_applies(const DecodeArgs& a);
+// The shape test of decode_umma_applies (a global layer's cache is contiguous and un-rotated).
+bool decode_umma_shape(const gemma_attn_params* p, int n_q);
 cudaError_t launch_decode_umma_any(const DecodeArgs& a, cudaStream_t stream);
 // 3-D bf16 tensor map over a decode cache [planes][capacity][d] with {64, 128, 1} boxes,
 // 128-byte swizzle.

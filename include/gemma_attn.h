@@ -280,7 +280,11 @@ int gemma_attn_decode_shard(const gemma_attn_params* params, const void* q, cons
                             int32_t max_shard_len, float* partial_o, float* partial_lse,
                             int32_t num_splits, void* stream);
 
-/* A split count for gemma_attn_decode that fills the GPU for this shape. */
+/* A split count for gemma_attn_decode that fills the GPU for this shape. For the shapes
+ * of the tcgen05 verify kernel (a GLOBAL layer, head dim 256 or 512, 9..32 query rows per
+ * KV head) it is twice the uniform-length choice, at most one split per 128 keys: that
+ * kernel sizes its work items from the actual lengths and uses at most this many splits
+ * per sequence. */
 int gemma_attn_decode_num_splits(const gemma_attn_params* params, int32_t batch, int32_t n_q,
                                  int32_t max_cache_len, int32_t* num_splits);
 

@@ -205,6 +205,22 @@ def test_decode_split_hint():
     assert G.gemma_attn_decode_num_splits(loc, 8, 1, 5) == 1
 
 
+def test_decode_split_hint_verify_shapes(monkeypatch):
+    # the tcgen05 verify kernel's shapes (global, 9..32 rows per KV head) get twice the
+    # uniform-length choice, at most one split per 128 keys; the legacy path keeps it
+    glo = _p(kind=G.GLOBAL, num_q_heads=32, num_kv_heads=4, head_dim=512, rope_p=0.25)
+    for batch, n_q, max_len in [(16, 4, 42740), (2, 4, 300), (8, 2, 131072)]:
+        monkeypatch.setenv("GEMMA_ATTN_DECODE_MMA_SYNC", "1")
+        uniform = G.gemma_attn_decode_num_splits(glo, batch, n_q, max_len)
+        monkeypatch.delenv("GEMMA_ATTN_DECODE_MMA_SYNC")
+        got = G.gemma_attn_decode_num_splits(glo, batch, n_q, max_len)
+        assert got == min(2 * uniform, (max_len + n_q + 127) // 128)
+    # 8 rows per KV head stay on the warp kernel: no doubling
+    one = G.gemma_attn_decode_num_splits(glo, 8, 1, 131072)
+    monkeypatch.setenv("GEMMA_ATTN_DECODE_MMA_SYNC", "1")
+    assert G.gemma_attn_decode_num_splits(glo, 8, 1, 131072) == one
+
+
 def test_shard_entry_point_argument_rules():
     # rejected before any launch: no device is needed
     loc = G.params(G.LOCAL, 8, 4, 256, window=64)

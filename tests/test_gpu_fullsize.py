@@ -123,11 +123,14 @@ def test_ragged_prefill_both_kinds():
         _prefill_case(layer, pre.seq_lens, seed=300 + li, rows=rows)
 
 
-def _decode_case(layer: W.LayerSpec, cache_lens, n_q, seed, check_batches=(0,)):
-    """Full-size decode/verify; checks query heads of KV head 0 for the given sequences."""
+def _decode_case(layer: W.LayerSpec, cache_lens, n_q, seed, check_batches=(0,), all_heads=False):
+    """Full-size decode/verify; checks the query heads of KV head 0 (every KV head with
+    all_heads) for the given sequences."""
     B = len(cache_lens)
     Hq, Hkv, d = layer.num_q_heads, layer.num_kv_heads, layer.head_dim
     group = Hq // Hkv
+    hk = Hkv if all_heads else 1      # KV heads and query heads with oracle-visible data
+    hq = Hq if all_heads else group
     max_len = max(cache_lens)
     local = layer.kind == W.LOCAL
     cap = layer.window if local else max_len
@@ -146,21 +149,21 @@ def _decode_case(layer: W.LayerSpec, cache_lens, n_q, seed, check_batches=(0,)):
     hists = {}
     for b in check_batches:
         n = cache_lens[b]
-        kh = W.normal_bf16(seed + b, 1, (n + n_q, 1, d))
-        vh = None if layer.k_eq_v else W.normal_bf16(seed + b, 2, (n + n_q, 1, d))
-        qb = W.normal_bf16(seed + b, 0, (1, n_q, group, d))
+        kh = W.normal_bf16(seed + b, 1, (n + n_q, hk, d))
+        vh = None if layer.k_eq_v else W.normal_bf16(seed + b, 2, (n + n_q, hk, d))
+        qb = W.normal_bf16(seed + b, 0, (1, n_q, hq, d))
         hists[b] = (kh, vh, qb)
-        q[b, :, 0:group] = dev_bf16(qb[0])
-        nk[b, :, 0] = dev_bf16(kh[n:, 0])
+        q[b, :, 0:hq] = dev_bf16(qb[0])
+        nk[b, :, 0:hk] = dev_bf16(kh[n:])
         if nv is not None:
-            nv[b, :, 0] = dev_bf16(vh[n:, 0])
+            nv[b, :, 0:hk] = dev_bf16(vh[n:])
         if local:
             lo = max(0, n - cap)
             slots = torch.from_numpy(np.arange(lo, n) % cap).cuda()
-            kc[b, 0, slots] = dev_bf16(kh[lo:n, 0])
-            vc[b, 0, slots] = dev_bf16(vh[lo:n, 0])
+            kc[b, 0:hk, slots] = dev_bf16(kh[lo:n]).transpose(0, 1)
+            vc[b, 0:hk, slots] = dev_bf16(vh[lo:n]).transpose(0, 1)
         else:
-            kc[b, 0, :n] = dev_bf16(kh[:n, 0])
+            kc[b, 0:hk, :n] = dev_bf16(kh[:n]).transpose(0, 1)
     p = G.params(layer.kind, Hq, Hkv, d, window=layer.window, rope_p=layer.rope_p, rope_base=layer.rope_base,
                  softmax_scale=layer.softmax_scale)
     splits = G.gemma_attn_decode_num_splits(p, B, n_q, max_len)
@@ -178,7 +181,7 @@ def _decode_case(layer: W.LayerSpec, cache_lens, n_q, seed, check_batches=(0,)):
         kh, vh, qb = hists[b]
         ref, _ = oracle.decode(layer.kind, layer.window, layer.rope_p, layer.rope_base, layer.softmax_scale,
                                qb, [kh], None if vh is None else [vh], [cache_lens[b]])
-        assert_close(got_all[b:b + 1, :, 0:group], ref, f"full-size decode {layer} b={b}")
+        assert_close(got_all[b:b + 1, :, 0:hq], ref, f"full-size decode {layer} b={b}")
 
 
 def test_long_context_decode_global():
@@ -195,3 +198,14 @@ def test_ragged_verify_both_kinds():
     _, ver = W.ragged_31b()
     for li, layer in enumerate(ver.layers):
         _decode_case(layer, list(ver.cache_lens), ver.n_q, seed=500 + li, check_batches=(0, 1, 7))
+
+
+def test_ragged_verify_global_every_kv_head():
+    """The tcgen05 verify kernel at full size: every KV head's group (CTAs of every
+    blockIdx.y), on the longest sequence and a short one."""
+    _, ver = W.ragged_31b()
+    layer = [l for l in ver.layers if l.kind == W.GLOBAL][0]
+    lens = list(ver.cache_lens)
+    b_long = int(np.argmax(lens))
+    b_short = int(np.argmin(lens))
+    _decode_case(layer, lens, ver.n_q, seed=520, check_batches=(b_long, b_short), all_heads=True)
