@@ -365,6 +365,38 @@ def test_combine_against_oracle():
     np.testing.assert_allclose(got_lse[np.isfinite(ref_lse)], ref_lse[np.isfinite(ref_lse)], atol=1e-5)
 
 
+@pytest.mark.parametrize("S,R,d", [(5, 37, 64), (18, 2048, 512), (3, 2100, 36), (2, 4096, 32)])
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_combine_vector_and_element_forms_agree(S, R, d, out_dtype):
+    # 16-byte aligned buffers with at least 2048 warps of work (rows x ceil(d / 128)) take
+    # the vectorized kernel (a warp per 128 columns of a row); buffers one element off, or
+    # fewer rows, take the per-element kernel. Both merge in split order, so the outputs
+    # are identical bit for bit, and both match the oracle.
+    rng = np.random.default_rng(S * 1000 + R)
+    po = rng.standard_normal((S, R, d)).astype(np.float32)
+    pl = (rng.standard_normal((S, R)) * 3).astype(np.float32)
+    pl[S - 1, : R // 2] = -np.inf
+    pl[:, R // 3] = -np.inf
+    f32 = out_dtype == "f32"
+    flag = G.OUT_F32 if f32 else G.OUT_BF16
+    tdt = torch.float32 if f32 else torch.bfloat16
+    pl_d = torch.from_numpy(pl).cuda()
+    outs = []
+    for off in (0, 1):
+        po_buf = torch.empty(S * R * d + 1, dtype=torch.float32, device="cuda")
+        po_buf[off:off + S * R * d] = torch.from_numpy(po.reshape(-1)).cuda()
+        out_buf = torch.full((R * d + 1,), 7.0, dtype=tdt, device="cuda")
+        lse = torch.empty((R,), dtype=torch.float32, device="cuda")
+        G.gemma_attn_combine(po_buf[off:], pl_d, S, R, d, flag, out_buf[off:], lse)
+        torch.cuda.synchronize()
+        outs.append((out_buf[off:off + R * d].float().cpu().numpy().reshape(R, d), lse.cpu().numpy()))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    ref, _ = oracle.combine(po.astype(np.float64), pl.astype(np.float64))
+    if f32:
+        assert_close(outs[0][0], ref, "combine vector form")
+
+
 def test_prefill_divergent_rescale_within_warp():
     """One key with a huge score: rows at or after it raise their running max by far more
     than 2^8 mid-sequence, rows before it do not, so lanes of one warp disagree."""
