@@ -111,6 +111,26 @@ def test_decode_argument_errors():
     assert e.value.status == G.ERR_UNSUPPORTED
 
 
+def test_combine_argument_errors():
+    fake = 1 << 20
+    bad = [
+        (0, fake, 2, 8, 64, G.OUT_BF16, fake),      # no partial_o
+        (fake, 0, 2, 8, 64, G.OUT_BF16, fake),      # no partial_lse
+        (fake, fake, 2, 8, 64, G.OUT_BF16, 0),      # no out
+        (fake, fake, 0, 8, 64, G.OUT_BF16, fake),   # no split
+        (fake, fake, 2, -1, 64, G.OUT_BF16, fake),  # negative row count
+        (fake, fake, 2, 8, 0, G.OUT_BF16, fake),    # empty head dim
+        (fake, fake, 2, 8, 64, 7, fake),            # unknown output type
+    ]
+    for po, pl, s, rows, d, dt, out in bad:
+        with pytest.raises(G.GemmaAttnError) as e:
+            G.gemma_attn_combine(po, pl, s, rows, d, dt, out, None)
+        assert e.value.status == G.ERR_INVALID_ARG
+    # no rows: nothing to merge, nothing launched
+    G.gemma_attn_combine(fake, fake, 2, 0, 64, G.OUT_F32, fake, None)
+    assert G.gemma_attn_last_launch_count() == 0
+
+
 def test_cache_append_argument_errors():
     p = _p(window=64)
     fake = 1 << 20
