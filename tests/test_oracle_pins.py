@@ -330,6 +330,12 @@ def test_combine_closed_form():
     assert abs(l[0] - math.log(4.0)) < 1e-15
     o, l = oracle.combine(np.zeros((2, 1, 2)), np.full((2, 1), -np.inf))
     assert l[0] == -np.inf and np.all(o == 0)
+    # the weights depend on lse differences only: a common shift by +-1e4 (exp of which
+    # overflows or underflows fp64) leaves the merge unchanged and shifts the lse
+    for shift in (1e4, -1e4):
+        o, l = oracle.combine(po, pl + shift)
+        np.testing.assert_allclose(o, [[1.0, 6.0]], atol=1e-12)
+        assert abs(l[0] - (shift + math.log(4.0))) < 1e-9
 
 
 def test_decode_equals_prefill_rows():
